@@ -174,6 +174,9 @@ bool choose_idx_plan(int H_I, int d_I, ic_dtype qk, int n_q, IdxPlan* pl) {
     return false;
 }
 
+// The top-k plus the keys of one append step must fit a query's candidate list.
+bool plan_supports_topk(const IdxPlan& pl, int topk) { return topk + pl.step_keys <= pl.C && topk <= 2048; }
+
 constexpr int MERGE_E = 32;              // merge kernel: up to 256 * 32 candidates per row
 constexpr int MERGE_MAX = 256 * MERGE_E;
 
@@ -242,7 +245,7 @@ ic_status launch_indexer(const void* q_I, const float* q_scale, const void* w, i
     if (batch == 0 || n_q == 0) return IC_OK;
     IdxPlan pl;
     if (!choose_idx_plan(H_I, d_I, qk_dt, n_q, &pl)) return IC_ERR_UNSUPPORTED;
-    if (topk + pl.step_keys > pl.C || topk > 2048) return IC_ERR_UNSUPPORTED;
+    if (!plan_supports_topk(pl, topk)) return IC_ERR_UNSUPPORTED;
     const DeviceInfo dev = device_info();
     if (dev.sms <= 0) return cuda_fail("device query", cudaErrorNoDevice);
     const IdxLayout L = idx_layout(pl, batch, n_q, n_k, topk, dev.sms, allow_dense);
@@ -657,7 +660,7 @@ ic_status ic_indexer_workspace_size(int batch, int n_q, int n_k, int H_I, int d_
     *bytes_out = 0;
     if (batch == 0 || n_q == 0) return IC_OK;
     IdxPlan pl;
-    if (!choose_idx_plan(H_I, d_I, qk_dtype, n_q, &pl)) return IC_ERR_UNSUPPORTED;
+    if (!choose_idx_plan(H_I, d_I, qk_dtype, n_q, &pl) || !plan_supports_topk(pl, topk)) return IC_ERR_UNSUPPORTED;
     const DeviceInfo dev = device_info();
     if (dev.sms <= 0) return cuda_fail("device query", cudaErrorNoDevice);
     *bytes_out = idx_layout(pl, batch, n_q, n_k, topk, dev.sms).bytes;
@@ -1098,7 +1101,7 @@ ic_status ic_indexer_topk_noalloc(const void* q_I, const float* q_scale, const v
     if (st != IC_OK) return st;
     if (batch == 0 || n_q == 0) return IC_OK;
     IdxPlan pl;
-    if (!choose_idx_plan(H_I, d_I, qk_dtype, n_q, &pl)) return IC_ERR_UNSUPPORTED;
+    if (!choose_idx_plan(H_I, d_I, qk_dtype, n_q, &pl) || !plan_supports_topk(pl, topk)) return IC_ERR_UNSUPPORTED;
     const DeviceInfo dev = device_info();
     if (dev.sms <= 0) return cuda_fail("device query", cudaErrorNoDevice);
     // the split candidate lists, not the decode score rows: their size does
@@ -1128,7 +1131,7 @@ ic_status ic_indexer_noalloc_scratch_size(int batch, int n_q, int n_k, int H_I, 
     *bytes_out = 0;
     if (batch == 0 || n_q == 0) return IC_OK;
     IdxPlan pl;
-    if (!choose_idx_plan(H_I, d_I, qk_dtype, n_q, &pl)) return IC_ERR_UNSUPPORTED;
+    if (!choose_idx_plan(H_I, d_I, qk_dtype, n_q, &pl) || !plan_supports_topk(pl, topk)) return IC_ERR_UNSUPPORTED;
     const DeviceInfo dev = device_info();
     if (dev.sms <= 0) return cuda_fail("device query", cudaErrorNoDevice);
     *bytes_out = idx_layout(pl, batch, n_q, n_k, topk, dev.sms, false).bytes;

@@ -98,6 +98,11 @@ ic_status ic_resolve_pattern(int n_layers, int index_topk_freq, const char* inde
  *   k_I     [batch, n_k, d_I]  qk_dtype
  *   k_scale [batch, n_k]  fp32 per-token scale of k_I (NULL for bf16;
  *           required and > 0 for FP8)
+ *           The scales live in device memory and are NOT checked: the host
+ *           never reads them (that would need a copy and a synchronisation).
+ *           A scale that is zero, negative or not finite breaks the
+ *           factoring of the scales out of the ReLU, and the selected keys
+ *           are then unspecified (no fault, no error status).
  *   idx_out [batch, n_q, topk] int32: for each query the indices of its top-k
  *           keys, in ASCENDING key-index order, followed by -1 entries when
  *           fewer than topk keys are visible. Which keys are selected is

@@ -37,8 +37,19 @@ def test_flop_counts_match_the_oracle(wl):
     compulsory, gather = bench.attn_bytes(wl)
     assert gather == keys * wl.d_qk * 2
     rows = wl.batch * wl.n_q
-    assert compulsory == (rows * wl.H * wl.d_qk * 2 + wl.batch * wl.n_k * wl.d_qk * 2 + rows * wl.topk * 4
+    # distinct KV rows the attention must read: the union of each sequence's
+    # index rows, bounded by min(n_k, that sequence's selected keys)
+    sel = idx.reshape(wl.batch, wl.n_q * wl.topk)
+    distinct = sum(len(np.unique(r[r >= 0])) for r in sel)
+    bound = wl.batch * min(wl.n_k, keys // wl.batch)
+    assert distinct <= bound
+    assert compulsory == (rows * wl.H * wl.d_qk * 2 + bound * wl.d_qk * 2 + rows * wl.topk * 4
                           + rows * wl.H * wl.d_v * 2)
+    if wl.n_q == 1:
+        assert distinct == bound          # decode: every selected row is distinct
+    else:
+        # causal prefill: almost every visible key is some query's choice
+        assert distinct >= 0.9 * min(wl.n_k, wl.q_pos0 + wl.n_q)
 
 
 def test_fp32_peak_is_derived_from_unit_counts_and_clock():

@@ -75,11 +75,19 @@ def test_noalloc_array_covers_every_supported_decode_shape(cuda_ok):
     lib.ic_indexer_noalloc_scratch_size.argtypes = [ctypes.c_int] * 7 + [ctypes.POINTER(ctypes.c_size_t)]
     lib.ic_indexer_noalloc_scratch_size.restype = ctypes.c_int
 
-    def need(b):
+    def need(b, H_I, d_I, topk, dt, n_k=32768):
         out = ctypes.c_size_t(0)
-        assert lib.ic_indexer_noalloc_scratch_size(b, 1, 32768, 64, 128, 2048, ic.FP8_E4M3,
+        assert lib.ic_indexer_noalloc_scratch_size(b, 1, n_k, H_I, d_I, topk, dt,
                                                    ctypes.byref(out)) == 0
         return out.value
 
-    worst = max(need(b) for b in range(1, 600))
-    assert 0 < worst <= limit
+    # every compiled decode plan at its largest supported top-k
+    for H_I, d_I, topk, dt in ((64, 128, 2048, ic.FP8_E4M3), (64, 128, 2048, ic.BF16),
+                               (4, 64, 128, ic.BF16)):
+        worst = max(need(b, H_I, d_I, topk, dt) for b in range(1, 600))
+        assert 0 < worst <= limit, (H_I, d_I, topk, dt, worst)
+
+    # a top-k the plan cannot serve is refused as unsupported, before sizing
+    out = ctypes.c_size_t(0)
+    assert lib.ic_indexer_noalloc_scratch_size(1, 1, 32768, 4, 64, 1024, ic.BF16,
+                                               ctypes.byref(out)) == 3
