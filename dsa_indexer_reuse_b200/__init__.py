@@ -14,7 +14,8 @@ Entry points (same names as the C ABI, without the ``ic_`` prefix):
     indexer_workspace_size, sparse_attn_workspace_size,
     layer_stack_workspace_size, get_device_status, debug_expire_wait,
     topk_overlap, search_pattern, greedy_pattern (pattern tools), and
-    overlap_matrix (layer x layer ratios from topk_overlap), and
+    overlap_matrix (layer x layer ratios), pattern_score (the search
+    objective of one pattern), and
     distill_target (the multi-layer distillation target and KL of one Full layer).
 The submodule ``workloads`` (seeded synthetic inputs) needs no library.
 """
@@ -24,7 +25,7 @@ _EXPORTS = (
     "get_device_status", "indexer_topk", "indexer_workspace_size", "layer_stack",
     "layer_stack_workspace_size", "lib", "resolve_pattern", "sparse_attn",
     "sparse_attn_workspace_size", "version", "topk_overlap", "overlap_matrix", "search_pattern",
-    "greedy_pattern", "StackHostCall", "layer_stack_host", "distill_target",
+    "greedy_pattern", "pattern_score", "StackHostCall", "layer_stack_host", "distill_target",
 )
 
 

@@ -96,6 +96,12 @@ lib.ic_debug_expire_wait.argtypes = [ctypes.c_longlong, _P]
 lib.ic_debug_expire_wait.restype = _I
 lib.ic_topk_overlap.argtypes = [_P, _P, _I, _I, _I, _P, _P]
 lib.ic_topk_overlap.restype = _I
+lib.ic_overlap_matrix_workspace_size.argtypes = [_I, ctypes.POINTER(_SZ)]
+lib.ic_overlap_matrix_workspace_size.restype = _I
+lib.ic_overlap_matrix.argtypes = [_P, _I, _I, _I, _I, _P, _SZ, _P, _P]
+lib.ic_overlap_matrix.restype = _I
+lib.ic_pattern_score.argtypes = [_P, _I, ctypes.c_char_p, ctypes.POINTER(ctypes.c_double)]
+lib.ic_pattern_score.restype = _I
 lib.ic_search_pattern.argtypes = [_P, _I, _I, ctypes.c_char_p, ctypes.POINTER(ctypes.c_double)]
 lib.ic_search_pattern.restype = _I
 _OBJECTIVE = ctypes.CFUNCTYPE(ctypes.c_double, ctypes.c_char_p, _P)
@@ -388,20 +394,39 @@ def topk_overlap(idx_a, idx_b, n_k: int, *, counts_out=None, stream=None):
 
 
 def overlap_matrix(idx_layers, n_k: int, stream=None) -> np.ndarray:
-    """Layer x layer overlap ratios from each layer's own index tensor:
-    R[a][b] = sum_rows |T_a & T_b| / sum_rows |T_a| (the share of layer a's
-    selections that layer b also selects). Runs ic_topk_overlap per pair."""
+    """Layer x layer overlap ratios from each layer's own index tensor
+    (ic_overlap_matrix): R[a][b] = sum_rows |T_a & T_b| / sum_rows |T_a|, the
+    share of layer a's selections that layer b also selects. Synchronises
+    the stream."""
     n = len(idx_layers)
-    valid = [torch.count_nonzero((t >= 0) & (t < n_k)).item() for t in idx_layers]
+    if n == 0:
+        raise ValueError("no index tensors")
+    _dev(*idx_layers)
+    shape = idx_layers[0].shape
+    if any(t.shape != shape or t.dtype != torch.int32 for t in idx_layers):
+        raise ValueError("index tensors must be int32 of one shape")
+    topk = shape[-1]
+    rows = idx_layers[0].numel() // max(topk, 1)
+    size = _SZ(0)
+    _check(lib.ic_overlap_matrix_workspace_size(n, ctypes.byref(size)), "ic_overlap_matrix_workspace_size")
+    ws = torch.empty(int(size.value), dtype=torch.uint8, device=idx_layers[0].device)
+    ptrs = (ctypes.c_void_p * n)(*[t.data_ptr() for t in idx_layers])
     R = np.zeros((n, n), np.float64)
-    for a in range(n):
-        for b in range(n):
-            if a == b:
-                R[a, b] = 1.0
-                continue
-            c = topk_overlap(idx_layers[a], idx_layers[b], n_k, stream=stream)
-            R[a, b] = c.sum().item() / max(valid[a], 1)
+    _check(lib.ic_overlap_matrix(ptrs, n, rows, topk, int(n_k), _ptr(ws), ws.numel(), R.ctypes.data,
+                                 _stream(stream)), "ic_overlap_matrix")
     return R
+
+
+def pattern_score(overlap, pattern: str) -> float:
+    """The pattern-search objective of one F/S pattern (ic_pattern_score):
+    sum over layers of overlap[l][nearest Full layer at or before l]."""
+    m = np.ascontiguousarray(overlap, dtype=np.float64)
+    n = m.shape[0]
+    if m.shape != (n, n):
+        raise ValueError("overlap must be square")
+    out = ctypes.c_double(0.0)
+    _check(lib.ic_pattern_score(m.ctypes.data, n, pattern.encode(), ctypes.byref(out)), "ic_pattern_score")
+    return float(out.value)
 
 
 def search_pattern(overlap, n_full: int):

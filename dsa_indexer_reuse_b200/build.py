@@ -1,6 +1,12 @@
 """Build the sm_100a shared library libindexcache.so in-tree with nvcc.
 
-    python -m dsa_indexer_reuse_b200.build [--force] [--verbose]
+    python -m dsa_indexer_reuse_b200.build [--force] [--verbose] [--debug]
+
+--debug builds libindexcache_debug.so instead: the same kernels compiled with
+IC_DEBUG, which checks the indices that are in bounds by construction (list
+appends, select outputs, compacted index rows, gathered rows) and records
+IC_ERR_INTERNAL in the device status instead of accessing out of bounds.
+Load it with IC_LIB_PATH=<path> before importing the package.
 """
 
 from __future__ import annotations
@@ -14,6 +20,7 @@ SRC_DIR = os.path.join(HERE, "csrc")
 MAIN = os.path.join(SRC_DIR, "indexcache.cu")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include", "indexcache.h")
 LIB = os.path.join(HERE, "libindexcache.so")
+DEBUG_LIB = os.path.join(HERE, "libindexcache_debug.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -38,18 +45,19 @@ def nvcc_path() -> str:
     return "nvcc"
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and os.path.exists(LIB):
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    out = DEBUG_LIB if debug else LIB
+    if not force and os.path.exists(out):
         newest = max(os.path.getmtime(f) for f in _sources())
-        if os.path.getmtime(LIB) >= newest:
-            return LIB
-    tmp = LIB + ".tmp.%d" % os.getpid()
-    cmd = [nvcc_path(), *NVCC_FLAGS, *(["-Xptxas", "-v"] if verbose else []), "-o", tmp, MAIN]
+        if os.path.getmtime(out) >= newest:
+            return out
+    tmp = out + ".tmp.%d" % os.getpid()
+    cmd = [nvcc_path(), *NVCC_FLAGS, *(["-DIC_DEBUG"] if debug else []), *(["-Xptxas", "-v"] if verbose else []),
+           "-o", tmp, MAIN]
     subprocess.check_call(cmd, cwd=HERE)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="--verbose" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv, debug="--debug" in sys.argv))

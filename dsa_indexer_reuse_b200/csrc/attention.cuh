@@ -59,6 +59,7 @@ struct AttnParams {
     float sm_scale_log2;       // sm_scale * log2(e)
     int n_splits;
     int n_work;                // rows * n_splits
+    int prefetch_split;        // 1: L2-prefetch each slice's rows when its work item starts
 };
 
 template <int DQK_, int DV_>
@@ -268,7 +269,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             for (int u = 0; u < VPL; ++u) {
                 const bool ok = v[u] >= 0 && v[u] < p.n_k;
                 const uint32_t bal = __ballot_sync(0xffffffffu, ok);
-                if (ok) list_s[run + __popc(bal & lanemask_lt())] = v[u];
+                if (ok) {
+                    const int slot = run + __popc(bal & lanemask_lt());
+                    if (IC_DCHECK(slot < Cfg::MAX_TOPK)) list_s[slot] = v[u];
+                }
                 run += __popc(bal);
             }
             if (pw == 0 && lane == 0) cnt_s[0] = n_total;
@@ -293,6 +297,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 const int row_base = b * p.n_k;
                 const int fallback = list_s[lo];  // rows past the slice end re-read a valid row
                 const __nv_bfloat16* kvb = p.kv + static_cast<int64_t>(row_base) * Cfg::DQK;
+                if (p.prefetch_split) {
+                    // decode-style split: every selected row of this slice is asked of
+                    // L2 at once, so the slice's HBM reads run at full depth while the
+                    // tiles are gathered (from L2) and computed one after another
+                    for (int e = lo + ptid; e < hi; e += Cfg::NPROD)
+                        prefetch_l2_bulk(kvb + static_cast<int64_t>(list_s[e]) * Cfg::DQK, Cfg::DQK * 2);
+                }
                 for (int j = 0; j < n_tiles; ++j) {
                     const int s = kv_n & 1;
                     const bool issue = mbar_wait(bar_kv_empty(s), ((kv_n >> 1) & 1) ^ 1, abort_flag);
@@ -323,7 +334,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                         constexpr int UPL = (UPR + 31) / 32;
                         for (int rr = pw; rr < Cfg::BK; rr += NW) {
                             const int e = lo + j * Cfg::BK + rr;
-                            const int key = e < hi ? list_s[e] : fallback;
+                            int key = e < hi ? list_s[e] : fallback;
+                            if (!IC_DCHECK(key >= 0 && key < p.n_k)) key = 0;
                             const __nv_bfloat16* src = kvb + static_cast<int64_t>(key) * Cfg::DQK;
                             const uint32_t row_dst = tile + (rr >> 3) * 1024 + (rr & 7) * 128;
                             const int x = rr & 7;

@@ -16,7 +16,8 @@
 // construction (list counts never pass their capacity, select outputs never
 // pass k, compacted index rows hold only keys in [0, n_k)); the one count
 // read back from global memory (the split lists' lengths in the merge) is
-// checked, and a failed check records IC_ERR_INTERNAL.
+// checked, and a failed check records IC_ERR_INTERNAL. The IC_DEBUG build
+// checks the by-construction indices too (IC_DCHECK).
 #pragma once
 
 #include <cuda.h>
@@ -45,6 +46,17 @@ __device__ __forceinline__ bool in_bounds(bool ok) {
     if (__builtin_expect(!ok, 0)) record_status(IC_ERR_INTERNAL);
     return ok;
 }
+
+// Checks of indices that are in bounds by construction (list appends,
+// select outputs, compacted index rows, gathered rows). The release build
+// compiles them away; a build with -DIC_DEBUG (build.py --debug) evaluates
+// them like in_bounds: a failure records IC_ERR_INTERNAL and skips the
+// access, with no trap.
+#ifdef IC_DEBUG
+#define IC_DCHECK(cond) ::ic::in_bounds(cond)
+#else
+#define IC_DCHECK(cond) true
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -198,6 +210,13 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* tma
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(x), "r"(row0), "r"(row1), "r"(row2),
         "r"(row3)
         : "memory");
+}
+
+// Ask L2 to fetch `bytes` (a multiple of 16) at a 16-byte aligned global
+// address; no data reaches the SM and nothing waits for it.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+                 : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* tmap) {

@@ -147,7 +147,9 @@ IdxPlan idx_plan() {
     IdxPlan pl;
     pl.G = Cfg::G;
     pl.C = Cfg::C;
-    pl.step_keys = ic::IDX_BM * Cfg::PSTEP;
+    // room a list needs above topk: one append step (generic path); the FAST
+    // path's cut must leave the list below its high-water mark (topk + 3 tiles)
+    pl.step_keys = Cfg::FAST ? 3 * ic::IDX_BM : ic::IDX_BM * Cfg::PSTEP;
     pl.smem = Cfg::SMEM_ALLOC;
     pl.threads = Cfg::THREADS;
     pl.regs = Cfg::REGS_LAUNCH;
@@ -431,6 +433,10 @@ ic_status launch_attn(const void* q, const void* kv, const int32_t* idx, int bat
     p.sm_scale_log2 = sm_scale * 1.4426950408889634f;
     p.n_splits = splits;
     p.n_work = rows * splits;
+    // decode-style calls read their rows from HBM: every slice is prefetched into
+    // L2 up front when all the launch's selected rows fit in a part of L2
+    const double sel_bytes = static_cast<double>(rows) * topk * d_qk * 2;
+    p.prefetch_split = (splits > 1 && sel_bytes <= 80e6) ? 1 : 0;
     if (check_register_pool(pl.kernel, pl.regs) != IC_OK)
         return cuda_fail("attention register pool", cudaErrorInvalidConfiguration);
     cudaError_t e = cudaFuncSetAttribute(pl.kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
@@ -532,6 +538,72 @@ ic_status ic_topk_overlap(const int32_t* idx_a, const int32_t* idx_b, int rows, 
         idx_a, idx_b, rows, topk, n_k, counts_out);
     e = cudaGetLastError();
     return e == cudaSuccess ? IC_OK : cuda_fail("overlap launch", e);
+}
+
+ic_status ic_overlap_matrix_workspace_size(int n_layers, size_t* bytes_out) {
+    if (!bytes_out || n_layers < 1 || n_layers > ic::OVERLAP_MAX_LAYERS) return IC_ERR_INVALID_ARG;
+    *bytes_out = round_up(static_cast<size_t>(n_layers) * n_layers * sizeof(unsigned long long), 256);
+    return IC_OK;
+}
+
+ic_status ic_overlap_matrix(const int32_t* const* idx_layers, int n_layers, int rows, int topk, int n_k,
+                            void* workspace, size_t workspace_bytes, double* ratio_out, void* stream) {
+    if (!idx_layers || !ratio_out || n_layers < 1 || rows < 0 || topk <= 0 || n_k < 0) return IC_ERR_INVALID_ARG;
+    if (n_layers > ic::OVERLAP_MAX_LAYERS) return IC_ERR_UNSUPPORTED;
+    for (int l = 0; l < n_layers; ++l)
+        if (!idx_layers[l]) return IC_ERR_INVALID_ARG;
+    const size_t bits_bytes = static_cast<size_t>((std::max(n_k, 1) + 31) / 32) * 4;
+    if (bits_bytes > 224 * 1024) return IC_ERR_UNSUPPORTED;
+    const size_t need = static_cast<size_t>(n_layers) * n_layers * sizeof(unsigned long long);
+    if (!workspace || workspace_bytes < need) return IC_ERR_WORKSPACE;
+    const DeviceInfo dev = device_info();
+    if (dev.sms <= 0) return cuda_fail("device query", cudaErrorNoDevice);
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    unsigned long long* counts = static_cast<unsigned long long*>(workspace);
+    cudaError_t e = cudaMemsetAsync(counts, 0, need, cs);
+    if (e != cudaSuccess) return cuda_fail("overlap counts reset", e);
+    if (rows > 0) {
+        ic::OverlapLayers L{};
+        for (int l = 0; l < n_layers; ++l) L.p[l] = idx_layers[l];
+        e = cudaFuncSetAttribute(&ic::overlap_counts_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(bits_bytes));
+        if (e != cudaSuccess) return cuda_fail("overlap smem attribute", e);
+        const int grid = std::max(1, std::min(rows, dev.sms));
+        for (int a = 0; a < n_layers; ++a) {
+            ic::overlap_counts_kernel<<<grid, ic::OVERLAP_THREADS, bits_bytes, cs>>>(L, a, n_layers, rows, topk, n_k,
+                                                                                   counts);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return cuda_fail("overlap counts launch", e);
+        }
+    }
+    std::vector<unsigned long long> host(static_cast<size_t>(n_layers) * n_layers);
+    e = cudaMemcpyAsync(host.data(), counts, need, cudaMemcpyDeviceToHost, cs);
+    if (e != cudaSuccess) return cuda_fail("overlap counts copy", e);
+    e = cudaStreamSynchronize(cs);
+    if (e != cudaSuccess) return cuda_fail("overlap counts synchronize", e);
+    // R[a][b] = overlap counts over layer a's valid entries (the diagonal)
+    for (int a = 0; a < n_layers; ++a) {
+        const double valid = static_cast<double>(host[static_cast<size_t>(a) * n_layers + a]);
+        for (int b = 0; b < n_layers; ++b) {
+            const size_t i = static_cast<size_t>(a) * n_layers + b;
+            ratio_out[i] = a == b ? 1.0 : static_cast<double>(host[i]) / std::max(valid, 1.0);
+        }
+    }
+    return IC_OK;
+}
+
+ic_status ic_pattern_score(const double* overlap, int n_layers, const char* pattern, double* score_out) {
+    if (!overlap || !pattern || !score_out || n_layers < 1) return IC_ERR_INVALID_ARG;
+    if (std::strlen(pattern) != static_cast<size_t>(n_layers) || pattern[0] != 'F') return IC_ERR_BAD_PATTERN;
+    double s = 0.0;
+    int src = 0;
+    for (int l = 0; l < n_layers; ++l) {
+        if (pattern[l] == 'F') src = l;
+        else if (pattern[l] != 'S') return IC_ERR_BAD_PATTERN;
+        s += overlap[static_cast<size_t>(l) * n_layers + src];
+    }
+    *score_out = s;
+    return IC_OK;
 }
 
 ic_status ic_search_pattern(const double* overlap, int n_layers, int n_full, char* pattern_out, double* score_out) {

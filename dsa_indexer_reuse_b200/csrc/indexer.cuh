@@ -20,12 +20,21 @@
 //  * Epilogue: each thread owns one key (one TMEM lane) and reduces its
 //    heads in registers: ReLU, multiply by w, sum (packed f32x2 FMA), scale.
 //    The L x L score matrix never leaves the SM.
-//  * Streaming top-k: per query an append-only candidate list in shared
-//    memory, kept in ascending key order (ballot + per-warp counts, one
-//    warpgroup barrier per tile), admitting only scores above the query's
-//    threshold. A full list is cut back by block_select (value-bucket select +
-//    stable compaction), which raises the threshold. At the end an exact
-//    select writes the k winners in ascending key order, -1 padded.
+//  * Streaming top-k: per query a candidate list in shared memory that
+//    admits only keys ranked above the query's threshold. In the 64-head
+//    configurations (one query per epilogue warpgroup) every warp appends
+//    its passing keys with one shared-memory atomic per tile, without a
+//    barrier, and candidates are ranked by the composite (score, index) of
+//    topk_comp.cuh. The epilogue warps meet only at sync points, scheduled
+//    from the fullest list's free room (no list can overflow before the
+//    next one); at a sync point where some list is near capacity every
+//    warpgroup cuts its list (a sampled threshold, or the exact k-th
+//    composite), which raises its threshold. Other configurations keep ascending lists
+//    with one warpgroup barrier per tile (ballot + per-warp counts) and
+//    block_select cuts. At the end an exact select writes the k winners,
+//    -1 padded.
+//  * Rows that see no more than k keys select all of them: their work items
+//    write 0..t directly and skip the contraction.
 //  * Long-row first scheduling: work items (query group, key chunk) are
 //    ordered by decreasing length and dealt to persistent CTAs in a snake.
 //  * Decode-style calls (one query per sequence) split the key range into
@@ -36,7 +45,17 @@
 #pragma once
 
 #include "common.cuh"
+#include <type_traits>
+
+#include "topk_comp.cuh"
 #include "topk_select.cuh"
+
+// FAST epilogue: of the 8 column pairs of heads a thread reduces per key,
+// the first IC_IDX_RELU_REPS take max + packed FMA, the rest the |x| form
+// (see the epilogue); 8 keeps every head on the max form.
+#ifndef IC_IDX_RELU_REPS
+#define IC_IDX_RELU_REPS 8
+#endif
 
 namespace ic {
 
@@ -85,9 +104,16 @@ struct IdxCfg {
     static constexpr int REGS_EPI = REGS_EPI_RAW > 248 ? 248 : REGS_EPI_RAW;
     static_assert(128 * REGS_CTRL + 128 * NUM_EPI_WG * REGS_EPI <= REGS_LAUNCH * THREADS, "register split");
     static constexpr int C = 128 * E;              // candidate capacity per query
-    // 64-head, one-query-per-warpgroup configurations score two tiles per
-    // warpgroup barrier (one append step covers 256 keys)
-    static constexpr int PSTEP = (HI == 64 && QPW == 1) ? 2 : 1;
+    // 64-head configurations with one query per epilogue warpgroup use the
+    // barrier-free append and composite-ranked lists (topk_comp.cuh)
+    static constexpr bool FAST = (HI == 64 && QPW == 1);
+    static constexpr int PSTEP = 1;                // tiles per append step (generic path)
+    static constexpr int RELU_REPS = IC_IDX_RELU_REPS;
+    static_assert(RELU_REPS >= 0 && RELU_REPS <= 8, "RELU_REPS");
+    // FAST: keys one append step can add to a query's list (one tile); the
+    // plan needs topk + 2 steps of room so a cut always leaves a free step
+    static constexpr int STEP_KEYS = IDX_BM;
+    static constexpr int EPI_THREADS = 128 * NUM_EPI_WG;
     static constexpr int Q_BYTES = N * ROW_BYTES;
     static constexpr int K_BYTES = IDX_BM * ROW_BYTES;
     static constexpr int TMEM_COLS = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128
@@ -95,11 +121,13 @@ struct IdxCfg {
     static constexpr uint32_t IDESC = make_idesc(IDX_BM, N, FP8 ? FMT_E4M3 : FMT_BF16,
                                                  FP8 ? FMT_E4M3 : FMT_BF16);
     struct WGState {
-        int cnt[2][4][QPW * PSTEP];  // per-step ballot counts (tile, query), by step parity
-        int count[2][QPW];      // candidate counts, by tile parity
-        uint32_t thr[2][QPW];   // insertion thresholds, by tile parity
+        int cnt[2][4][QPW * PSTEP];  // generic: per-step ballot counts (tile, query), by step parity
+        int count[2][QPW];      // generic: candidate counts, by tile parity
+        uint32_t thr[2][QPW];   // generic: insertion thresholds, by tile parity
+        unsigned long long fthr;  // FAST: admission threshold (composite)
+        unsigned fcount;        // FAST: candidate count (atomic appends)
     };
-    using Scratch = SelectScratch<128, E>;
+    using Scratch = typename std::conditional<FAST, CompScratch<128, E>, SelectScratch<128, E>>::type;
     // shared memory layout (byte offsets)
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + Q_BYTES;
@@ -127,6 +155,7 @@ __device__ __forceinline__ float load_w(const IdxParams& p, int64_t i) {
 
 struct IdxWork {
     int b, q0, nq_valid, k_begin, k_end, n_tiles;
+    bool trivial;  // every query of the group sees at most topk keys: all are selected
 };
 
 template <class Cfg>
@@ -144,6 +173,10 @@ __device__ __forceinline__ IdxWork idx_work(const IdxParams& p, int item) {
     w.k_begin = c * p.chunk;
     w.k_end = min(n_vis, (c + 1) * p.chunk);
     w.n_tiles = w.k_end > w.k_begin ? ceil_div(w.k_end - w.k_begin, IDX_BM) : 0;
+    // the selection of a query that sees at most topk keys is all of them (no
+    // scores needed); only for direct output (split chunks feed the merge)
+    w.trivial = S == 1 && n_vis <= p.topk;
+    if (w.trivial) w.n_tiles = 0;
     return w;
 }
 
@@ -311,6 +344,18 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             if (item >= p.n_work) continue;
             const IdxWork wk = idx_work<Cfg>(p, item);
             const int c_split = item % p.n_splits;
+            if (wk.trivial) {
+                // every visible key is selected: 0..n_vis-1, then -1
+                for (int gl = 0; gl < QPW; ++gl) {
+                    const int g = e * QPW + gl;
+                    if (g >= wk.nq_valid) continue;
+                    const int64_t row = static_cast<int64_t>(wk.b) * p.n_q + wk.q0 + g;
+                    const int n_vis = max(0, min(p.q_pos0 + wk.q0 + g + 1, p.n_k));
+                    int32_t* out = p.idx_out + row * p.topk;
+                    for (int i = wtid; i < p.topk; i += 128) out[i] = i < n_vis ? i : -1;
+                }
+                continue;
+            }
             // per-query head weights, folded with the query's token scale
             for (int i = wtid; i < Cfg::COLS_PER_WG; i += 128) {
                 const int g = e * QPW + i / HI;
@@ -323,9 +368,16 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 }
                 w_s[g * HI + j] = v;
             }
-            for (int i = wtid; i < QPW; i += 128) {
-                st.count[par][i] = 0;
-                st.thr[par][i] = 0u;
+            if constexpr (Cfg::FAST) {
+                if (wtid == 0) {
+                    st.fcount = 0u;
+                    st.fthr = 0ull;
+                }
+            } else {
+                for (int i = wtid; i < QPW; i += 128) {
+                    st.count[par][i] = 0;
+                    st.thr[par][i] = 0u;
+                }
             }
             named_bar_sync(bar_id, 128);
 
@@ -335,7 +387,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             // shape: a thread holds 16 heads of 4 keys, so it reads only those 16
             // weights, and the 4 threads sharing the keys finish the sum with a
             // reduce-scatter that leaves key r + 8 i(c) in lane 4r + c.
-            constexpr bool FAST = (HI == 64 && QPW == 1);
+            constexpr bool FAST = Cfg::FAST;
             const int c4 = lane & 3, r8 = lane >> 2;
             const int kidx = FAST ? r8 + 8 * (2 * (c4 & 1) + (c4 >> 1)) : lane;
             // lanes whose key precedes this lane's key (for the in-order append)
@@ -353,6 +405,188 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                            : 1.f;
             };
             float ksc_next = key_scale(0);
+
+            if constexpr (FAST) {
+              // ---------------- 64 heads, one query per warpgroup: barrier-free append
+              uint32_t* ck = cand_key_s + e * C;
+              int32_t* ci = cand_idx_s + e * C;
+              auto load_key = [&](int pos) { return ck[pos]; };
+              auto load_id = [&](int pos) { return ci[pos]; };
+              auto comp_at = [&](int pos) { return comp_key(ck[pos], ci[pos]); };
+              const int pos_g = p.q_pos0 + wk.q0 + e;
+              uint64_t thr = 0ull;  // admission threshold; changes only in cuts
+              // The epilogue warps meet every `per` tiles. A list that an append
+              // left above `hw` since the last meeting makes every warpgroup cut
+              // its list there; otherwise every list is at most hw long, and the
+              // next `per` tiles (128 keys each) fit: no list ever overflows.
+              const int per = (Cfg::C - p.topk >= 10 * IDX_BM) ? 4 : 2;
+              const int hw = Cfg::C - per * IDX_BM;
+              bool crossed = false;  // lane 0: this warp left its list above hw since the last meeting
+              // TMEM -> registers: keys r, r+8 (ra) and r+16, r+24 (rb) of this
+              // warp's lane quarter, 16 heads each. The loads of tile t+1 are
+              // issued before the append of tile t, so their latency overlaps it.
+              uint32_t ra[32], rb[32];
+              auto issue_loads = [&](uint32_t it) {
+                  mbar_wait(bar_acc_full(it & 1), (it >> 1) & 1, abort_flag);
+                  tc_fence_after();
+                  const uint32_t tb = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + (it & 1) * Cfg::N +
+                                      e * Cfg::COLS_PER_WG;
+                  tmem_ld_16x256b_x8(tb, ra);
+                  tmem_ld_16x256b_x8(tb + (16u << 16), rb);
+              };
+              if (wk.n_tiles > 0) issue_loads(ait);
+              for (int t = 0; t < wk.n_tiles; ++t, ++ait) {
+                const int a = ait & 1;
+                // the next tile's key scale is requested a whole tile ahead
+                const float ksc = ksc_next;
+                ksc_next = key_scale(t + 1);
+                // this lane's 16 head weights (8-byte loads shared by the 8 lanes
+                // of a column pair)
+                float2 wreg[8];
+                const float* wg = w_s + e * HI + 2 * c4;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) wreg[i] = *reinterpret_cast<const float2*>(wg + 8 * i);
+                tmem_wait_ld();
+                // Heads of the first RELU_REPS column pairs: w . ReLU(x) (max on the
+                // ALU, packed FMA); the rest: w . ReLU(x) = (w.x + w.|x|) / 2 with |x|
+                // an FMA operand, which moves the work to the FMA pipe
+                float2 acc[4], lin[4];
+                float aab[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    acc[u] = make_float2(0.f, 0.f);
+                    lin[u] = make_float2(0.f, 0.f);
+                    aab[u] = 0.f;
+                }
+                auto relu2 = [](uint32_t x, uint32_t y) {
+                    return make_float2(fmaxf(__uint_as_float(x), 0.f), fmaxf(__uint_as_float(y), 0.f));
+                };
+                auto head_pair = [&](int i, uint32_t x, uint32_t y, int u) {
+                    if (i < Cfg::RELU_REPS) {
+                        acc[u] = __ffma2_rn(wreg[i], relu2(x, y), acc[u]);
+                    } else {
+                        lin[u] = __ffma2_rn(wreg[i], make_float2(__uint_as_float(x), __uint_as_float(y)), lin[u]);
+                        aab[u] = fmaf(wreg[i].x, fabsf(__uint_as_float(x)), aab[u]);
+                        aab[u] = fmaf(wreg[i].y, fabsf(__uint_as_float(y)), aab[u]);
+                    }
+                };
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    head_pair(i, ra[4 * i], ra[4 * i + 1], 0);      // key r
+                    head_pair(i, ra[4 * i + 2], ra[4 * i + 3], 1);  // key r + 8
+                    head_pair(i, rb[4 * i], rb[4 * i + 1], 2);      // key r + 16
+                    head_pair(i, rb[4 * i + 2], rb[4 * i + 3], 3);  // key r + 24
+                }
+                // the accumulator stage is free once read
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_acc_empty(a));
+                const bool meet = (t + 1) % per == 0 && t + 1 < wk.n_tiles;  // same in every epilogue thread
+                if (!meet && t + 1 < wk.n_tiles) issue_loads(ait + 1);
+                float pk[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    pk[u] = acc[u].x + acc[u].y;
+                    if (Cfg::RELU_REPS < 8) pk[u] += 0.5f * ((lin[u].x + lin[u].y) + aab[u]);
+                }
+                // reduce-scatter over the 4 lanes of a row: after the xor-1 step a
+                // lane holds keys {0,1} (even c) or {2,3} (odd c) of its row, after
+                // the xor-2 step one key
+                const bool odd = (c4 & 1) != 0;
+                const float q0 = (odd ? pk[2] : pk[0]) + __shfl_xor_sync(0xffffffffu, odd ? pk[0] : pk[2], 1);
+                const float q1 = (odd ? pk[3] : pk[1]) + __shfl_xor_sync(0xffffffffu, odd ? pk[1] : pk[3], 1);
+                const bool hi2 = (c4 & 2) != 0;
+                const float sum = (hi2 ? q1 : q0) + __shfl_xor_sync(0xffffffffu, hi2 ? q0 : q1, 2);
+                const uint32_t kk = float_to_ordered(sum * ksc);
+                const int s_key = wk.k_begin + t * IDX_BM + key_lane;
+                const bool valid = s_key < wk.k_end && e < wk.nq_valid && s_key <= pos_g;
+
+                // ---- append this tile's passing keys (one atomic per warp)
+                const bool pass = valid && comp_key(kk, s_key) > thr;
+                const uint32_t bal = __ballot_sync(0xffffffffu, pass);
+                if (bal != 0u) {
+                    unsigned base = 0u;
+                    if (lane == 0) {
+                        const unsigned nb = static_cast<unsigned>(__popc(bal));
+                        base = atomicAdd(&st.fcount, nb);
+                        crossed |= base + nb > static_cast<unsigned>(hw);
+                    }
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    if (pass) {
+                        const int pos = static_cast<int>(base) + __popc(bal & rank_mask);
+                        if (IC_DCHECK(pos < C)) {
+                            ck[pos] = kk;
+                            ci[pos] = s_key;
+                        }
+                    }
+                }
+
+                if (meet) {
+                    // ---- meeting: every list's appends so far are done; the OR says
+                    // whether any list passed hw
+                    const bool any = named_bar_or(5, Cfg::EPI_THREADS, crossed);
+                    crossed = false;
+                    if (any) {
+                        // every list past the middle of [topk, hw] is cut to its exact
+                        // top-k at this tile (the warpgroups stall together); a list
+                        // left uncut stays below hw
+                        const int n = static_cast<int>(st.fcount);  // same in the whole warpgroup
+                        if (n > (p.topk + hw) / 2) {
+                            const uint64_t tau =
+                                comp_select_kth<128, E>(n, p.topk, wtid, bar_id, sc, load_key, load_id);
+                            const int kept = comp_compact<128, E>(
+                                n, wtid, bar_id, sc, load_key, load_id, [&](int pos) { return comp_at(pos) >= tau; },
+                                [&](int o, uint32_t kv, int32_t iv) {
+                                    if (IC_DCHECK(o < n)) {
+                                        ck[o] = kv;
+                                        ci[o] = iv;
+                                    }
+                                });
+                            // no key ranked below tau can win: k kept keys rank at or above it
+                            if (wtid == 0) {
+                                st.fcount = static_cast<unsigned>(kept);
+                                st.fthr = tau;
+                            }
+                            named_bar_sync(bar_id, 128);
+                            thr = st.fthr;
+                        }
+                    }
+                    issue_loads(ait + 1);
+                }
+              }
+              // every warp's appends must be visible to the final select
+              named_bar_sync(bar_id, 128);
+              if (e < wk.nq_valid) {  // uniform across the warpgroup
+                  const int n = static_cast<int>(st.fcount);
+                  const int64_t row = static_cast<int64_t>(wk.b) * p.n_q + wk.q0 + e;
+                  uint64_t tau = 0ull;
+                  if (n > p.topk) tau = comp_select_kth<128, E>(n, p.topk, wtid, bar_id, sc, load_key, load_id);
+                  auto keep = [&](int pos) { return comp_at(pos) >= tau; };
+                  // warp wq appended keys with (s mod 128) in [32 wq, 32 wq + 32), in
+                  // ascending order: group-major emission is deterministic
+                  auto group = [&](int pos) { return (ci[pos] & (IDX_BM - 1)) >> 5; };
+                  if (p.n_splits == 1) {
+                      int32_t* out = p.idx_out + row * p.topk;
+                      const int kept = comp_emit_grouped<128, E>(n, wtid, bar_id, sc, keep, group, [&](int o, int pos) {
+                          if (IC_DCHECK(o < p.topk)) out[o] = ci[pos];
+                      });
+                      for (int i = kept + wtid; i < p.topk; i += 128) out[i] = -1;
+                  } else {
+                      const int64_t slot = row * p.n_splits + c_split;
+                      uint32_t* okey = p.cand_key + slot * p.topk;
+                      int32_t* oidx = p.cand_idx + slot * p.topk;
+                      const int kept = comp_emit_grouped<128, E>(n, wtid, bar_id, sc, keep, group,
+                                                                 [&](int o, int pos) {
+                                                                     if (IC_DCHECK(o < p.topk)) {
+                                                                         okey[o] = ck[pos];
+                                                                         oidx[o] = ci[pos];
+                                                                     }
+                                                                 });
+                      if (wtid == 0) p.cand_cnt[slot] = kept;
+                  }
+              }
+              named_bar_sync(bar_id, 128);
+            } else {
             constexpr int PS = Cfg::PSTEP;
             for (int t = 0; t < wk.n_tiles; t += PS) {
               // score PS tiles (releasing each accumulator stage as soon as it is
@@ -375,50 +609,6 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 tc_fence_after();
                 const int s_key = skey[sub];
                 const bool in_range = s_key < wk.k_end;
-                if constexpr (FAST) {
-                    // this lane's 16 head weights (8-byte loads shared by the 8 lanes
-                    // of a column pair; re-read per tile rather than held across the
-                    // list cuts)
-                    float2 wreg[8];
-                    const float* wg = w_s + e * HI + 2 * c4;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) wreg[i] = *reinterpret_cast<const float2*>(wg + 8 * i);
-                    uint32_t ra[32], rb[32];
-                    const uint32_t tb =
-                        tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + a * Cfg::N + e * Cfg::COLS_PER_WG;
-                    tmem_ld_16x256b_x8(tb, ra);
-                    tmem_ld_16x256b_x8(tb + (16u << 16), rb);
-                    tmem_wait_ld();
-                    float2 acc[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) acc[u] = make_float2(0.f, 0.f);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        auto relu2 = [](uint32_t x, uint32_t y) {
-                            return make_float2(fmaxf(__uint_as_float(x), 0.f), fmaxf(__uint_as_float(y), 0.f));
-                        };
-                        acc[0] = __ffma2_rn(wreg[i], relu2(ra[4 * i], ra[4 * i + 1]), acc[0]);      // key r
-                        acc[1] = __ffma2_rn(wreg[i], relu2(ra[4 * i + 2], ra[4 * i + 3]), acc[1]);  // key r + 8
-                        acc[2] = __ffma2_rn(wreg[i], relu2(rb[4 * i], rb[4 * i + 1]), acc[2]);      // key r + 16
-                        acc[3] = __ffma2_rn(wreg[i], relu2(rb[4 * i + 2], rb[4 * i + 3]), acc[3]);  // key r + 24
-                    }
-                    const float p0 = acc[0].x + acc[0].y, p1 = acc[1].x + acc[1].y;
-                    const float p2 = acc[2].x + acc[2].y, p3 = acc[3].x + acc[3].y;
-                    // reduce-scatter over the 4 lanes of a row: after the xor-1 step a
-                    // lane holds keys {0,1} (even c) or {2,3} (odd c) of its row, after
-                    // the xor-2 step one key
-                    const bool odd = (c4 & 1) != 0;
-                    const float q0 = (odd ? p2 : p0) + __shfl_xor_sync(0xffffffffu, odd ? p0 : p2, 1);
-                    const float q1 = (odd ? p3 : p1) + __shfl_xor_sync(0xffffffffu, odd ? p1 : p3, 1);
-                    const bool hi2 = (c4 & 2) != 0;
-                    const float sum = (hi2 ? q1 : q0) + __shfl_xor_sync(0xffffffffu, hi2 ? q0 : q1, 2);
-                    const float score = sum * ksc;
-                    const uint32_t kk = float_to_ordered(score);
-                    const int pos_g = p.q_pos0 + wk.q0 + e;
-                    const bool valid = in_range && e < wk.nq_valid && s_key <= pos_g;
-                    keyv[sub] = kk;
-                    if (valid && kk > st.thr[par][0]) passmask |= 1u << sub;
-                } else {
                 const uint32_t taddr =
                     tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + a * Cfg::N + e * Cfg::COLS_PER_WG;
 #pragma unroll
@@ -460,7 +650,6 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                         keyv[sub * QPW + gl] = kk;
                         if (valid && kk > st.thr[par][gl]) passmask |= 1u << (sub * QPW + gl);
                     }
-                }
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -521,8 +710,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                               [&](int pos) { return ci[pos]; }, [&](uint32_t k) { return k > tau; },
                               [&](int c) { return c >= p.topk && c <= hi; },
                               [&](int pos, uint32_t kv, int32_t iv) {
-                                  ck[pos] = kv;
-                                  ci[pos] = iv;
+                                  if (IC_DCHECK(pos < C)) {
+                                      ck[pos] = kv;
+                                      ci[pos] = iv;
+                                  }
                               });
                           if (kept >= 0) {
                               cnt_g = kept;
@@ -536,8 +727,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                               cnt_g, p.topk, false, relax, thr_g, wtid, bar_id, sc,
                               [&](int pos) { return ck[pos]; }, [&](int pos) { return ci[pos]; },
                               [&](int pos, uint32_t kv, int32_t iv) {
-                                  ck[pos] = kv;
-                                  ci[pos] = iv;
+                                  if (IC_DCHECK(pos < C)) {
+                                      ck[pos] = kv;
+                                      ci[pos] = iv;
+                                  }
                               });
                           cnt_g = sr.kept;
                           thr_g = sr.thr;
@@ -553,8 +746,10 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                           for (int q = 0; q < QPW * PS; ++q)
                               if (q == j) my_key = keyv[q];
                           const int pos = run + before[sub] + __popc(bal[j] & rank_mask);
-                          ck[pos] = my_key;
-                          ci[pos] = skey[sub];
+                          if (IC_DCHECK(pos < C)) {
+                              ck[pos] = my_key;
+                              ci[pos] = skey[sub];
+                          }
                       }
                       run += tot[sub];
                   }
@@ -583,7 +778,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                     int32_t* out = p.idx_out + row * p.topk;
                     const SelectResult sr = block_select<128, E>(
                         n, p.topk, true, p.topk, 0u, wtid, bar_id, sc, load_key, load_id,
-                        [&](int pos, uint32_t, int32_t iv) { out[pos] = iv; });
+                        [&](int pos, uint32_t, int32_t iv) {
+                            if (IC_DCHECK(pos < p.topk)) out[pos] = iv;
+                        });
                     for (int i = sr.kept + wtid; i < p.topk; i += 128) out[i] = -1;
                 } else {
                     const int64_t slot = row * p.n_splits + c_split;
@@ -592,13 +789,16 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                     const SelectResult sr = block_select<128, E>(
                         n, p.topk, true, p.topk, 0u, wtid, bar_id, sc, load_key, load_id,
                         [&](int pos, uint32_t kv, int32_t iv) {
-                            ok[pos] = kv;
-                            oi[pos] = iv;
+                            if (IC_DCHECK(pos < p.topk)) {
+                                ok[pos] = kv;
+                                oi[pos] = iv;
+                            }
                         });
                     if (wtid == 0) p.cand_cnt[slot] = sr.kept;
                 }
             }
             named_bar_sync(bar_id, 128);
+            }  // generic path
         }
     }
 
@@ -625,16 +825,17 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 }
 
 // Merge the per-chunk candidate lists of one query row into its final top-k
-// (used when the key range was split). One 256-thread CTA per row; chunk c's
-// list precedes chunk c+1's, so the concatenation is in ascending key order.
-// The lists are first copied into shared memory (dynamic: 8 bytes per
-// candidate, 256 * E candidates at most).
+// (used when the key range was split). One 256-thread CTA per row. The lists
+// are copied into shared memory one after the other (dynamic: 8 bytes per
+// candidate, 256 * E candidates at most); candidates are ranked by their
+// composite (score, index), so the order inside each list does not matter,
+// and the winners are written in the (deterministic) concatenated order.
 template <int E>
 __global__ void __launch_bounds__(256)
     topk_merge_kernel(const uint32_t* __restrict__ cand_key, const int32_t* __restrict__ cand_idx,
                       const int32_t* __restrict__ cand_cnt, int n_splits, int topk,
                       int32_t* __restrict__ idx_out) {
-    __shared__ SelectScratch<256, E> sc;
+    __shared__ CompScratch<256, E> sc;
     __shared__ int offs[17];
     extern __shared__ uint32_t merge_smem[];
     uint32_t* mkey = merge_smem;
@@ -663,11 +864,16 @@ __global__ void __launch_bounds__(256)
     __syncthreads();
     const int n = offs[n_splits];
     int32_t* out = idx_out + static_cast<int64_t>(row) * topk;
-    const SelectResult sr = block_select<256, E>(
-        n, topk, true, topk, 0u, tid, 1, sc, [&](int pos) { return mkey[pos]; },
-        [&](int pos) { return midx[pos]; },
-        [&](int pos, uint32_t, int32_t iv) { out[pos] = iv; });
-    for (int i = sr.kept + tid; i < topk; i += 256) out[i] = -1;
+    auto load_key = [&](int pos) { return mkey[pos]; };
+    auto load_id = [&](int pos) { return midx[pos]; };
+    uint64_t tau = 0ull;
+    if (n > topk) tau = comp_select_kth<256, E>(n, topk, tid, 1, sc, load_key, load_id);
+    const int kept = comp_compact<256, E>(
+        n, tid, 1, sc, load_key, load_id, [&](int pos) { return comp_key(mkey[pos], midx[pos]) >= tau; },
+        [&](int o, uint32_t, int32_t iv) {
+            if (IC_DCHECK(o < topk)) out[o] = iv;
+        });
+    for (int i = kept + tid; i < topk; i += 256) out[i] = -1;
 }
 
 }  // namespace ic

@@ -85,20 +85,11 @@ def main(argv=None):
     pat, score = ic.search_pattern(R, n_full)
     print("searched pattern (n_full=%d): %s  coverage %.4f of %d" % (n_full, pat, score, n))
     if args.objective == "coverage":
-        gpat, gval = ic.greedy_pattern(n, n_full, lambda p: -float(_coverage(R, p)))
+        gpat, gval = ic.greedy_pattern(n, n_full, lambda p: -ic.pattern_score(R, p))
         print("greedy pattern   (n_full=%d): %s  coverage %.4f of %d" % (n_full, gpat, -gval, n))
     else:
         gpat, gval = ic.greedy_pattern(n, n_full, attention_error_objective(wl, n))
         print("greedy pattern   (n_full=%d): %s  attention-output error %.4g vs all-Full" % (n_full, gpat, gval))
-
-
-def _coverage(R, pattern: str) -> float:
-    src, s = 0, 0.0
-    for l, c in enumerate(pattern):
-        if c == "F":
-            src = l
-        s += R[l, src]
-    return s
 
 
 if __name__ == "__main__":

@@ -104,11 +104,16 @@ ic_status ic_resolve_pattern(int n_layers, int index_topk_freq, const char* inde
  *           factoring of the scales out of the ReLU, and the selected keys
  *           are then unspecified (no fault, no error status).
  *   idx_out [batch, n_q, topk] int32: for each query the indices of its top-k
- *           keys, in ASCENDING key-index order, followed by -1 entries when
- *           fewer than topk keys are visible. Which keys are selected is
- *           exact: score descending, equal scores broken toward the lower key
- *           index (and -0.0 == +0.0). Scores are computed in fp32 from fp32
- *           tensor-core accumulators.
+ *           keys, each once, followed by -1 entries when fewer than topk keys
+ *           are visible. Which keys are selected is exact: score descending,
+ *           equal scores broken toward the lower key index (and -0.0 ==
+ *           +0.0). Scores are computed in fp32 from fp32 tensor-core
+ *           accumulators. The order of a row's entries is deterministic (the
+ *           same inputs give the same bytes) but otherwise unspecified: a
+ *           query that sees at most topk keys lists 0..t; H_I = 4 shapes and
+ *           decode score rows list ascending indices; the other 64-head
+ *           paths list the keys grouped by (index mod 128) / 32, ascending
+ *           within a group. Consumers treat a row as a set.
  * Supported shapes: H_I in {4, 64} (d_I = 64 for H_I = 4, 128 for H_I = 64),
  * FP8 only with d_I = 128, 1 <= topk <= 2048. Others: IC_ERR_UNSUPPORTED.
  * Workspace: ic_indexer_workspace_size (0 bytes for prefill; decode-style
@@ -301,6 +306,32 @@ ic_status ic_distill_target(const void* const* q_layers, const void* const* kv_l
  */
 ic_status ic_topk_overlap(const int32_t* idx_a, const int32_t* idx_b, int rows, int topk, int n_k,
                           int32_t* counts_out, void* stream);
+
+/*
+ * ic_overlap_matrix: the layer x layer overlap-ratio matrix of n_layers index
+ * buffers (each layer run with its own indexer), written to the host array
+ * ratio_out (row-major n_layers x n_layers, doubles):
+ *     ratio_out[a][b] = sum_r |valid(T_a[r]) & valid(T_b[r])| / sum_r |valid(T_a[r])|
+ * (the share of layer a's selections that layer b also selects; 1 on the
+ * diagonal, 0 rows when layer a selects nothing). idx_layers is a HOST array
+ * of n_layers device pointers, each [rows, topk] int32 as ic_indexer_topk
+ * writes it. Validity and the n_k limit as for ic_topk_overlap; n_layers <=
+ * 128, else IC_ERR_UNSUPPORTED. The counts accumulate in the caller's device
+ * workspace (ic_overlap_matrix_workspace_size bytes, else
+ * IC_ERR_WORKSPACE). Enqueued on `stream`, then the call synchronises that
+ * stream to read the counts back and returns with ratio_out filled.
+ */
+ic_status ic_overlap_matrix_workspace_size(int n_layers, size_t* bytes_out);
+ic_status ic_overlap_matrix(const int32_t* const* idx_layers, int n_layers, int rows, int topk, int n_k,
+                            void* workspace, size_t workspace_bytes, double* ratio_out, void* stream);
+
+/*
+ * ic_pattern_score (host only): the objective ic_search_pattern maximises,
+ * for one pattern: sum over layers l of overlap[l * n_layers + src(l)], with
+ * src(l) the nearest Full layer at or before l. `pattern` is n_layers
+ * characters 'F'/'S' starting with 'F' (else IC_ERR_BAD_PATTERN).
+ */
+ic_status ic_pattern_score(const double* overlap, int n_layers, const char* pattern, double* score_out);
 
 /*
  * ic_search_pattern (host only): the F/S pattern with exactly n_full Full

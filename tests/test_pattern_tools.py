@@ -138,3 +138,17 @@ def test_pattern_tools_reject_bad_arguments(ic):
         ic.greedy_pattern(4, 2, lambda p: float("inf"))
     with pytest.raises(ZeroDivisionError):
         ic.greedy_pattern(4, 2, lambda p: 1 / 0)
+
+
+@pytest.mark.parametrize("n", [1, 4, 9])
+def test_pattern_score_matches_oracle(ic, n):
+    rng = np.random.default_rng(n)
+    R = rng.random((n, n))
+    for bits in itertools.product("FS", repeat=n - 1):
+        pat = "F" + "".join(bits)
+        assert ic.pattern_score(R, pat) == pytest.approx(oracle.pattern_score(R, pat), rel=1e-15, abs=1e-15)
+    with pytest.raises(ic.IcError) as e:
+        ic.pattern_score(R, "S" * n)
+    assert e.value.code == 2
+    with pytest.raises(ic.IcError):
+        ic.pattern_score(R, "F" * (n + 1))

@@ -16,6 +16,7 @@ import pytest
 import torch
 
 from dsa_indexer_reuse_b200 import workloads as W
+from gpu_util import canon
 
 pytestmark = pytest.mark.gpu
 
@@ -59,9 +60,10 @@ def test_noalloc_matches_workspace_entry_point_twice(cuda_ok, wl):
         out = torch.full((wl.batch, wl.n_q, wl.topk), -7, dtype=torch.int32, device="cuda")
         assert _call_noalloc(lib, ic, d, wl, out) == 0
         torch.cuda.synchronize()
-        # index sets are exact (the tolerance the indexer tests use for
-        # identical inputs through the same kernels)
-        assert np.array_equal(out.cpu().numpy(), ref)
+        # index sets are exact: both paths score every key with the same
+        # arithmetic; the order of a row's entries may differ between the
+        # split lists and the score-row select, so rows compare as sets
+        assert np.array_equal(canon(out.cpu().numpy().reshape(-1, wl.topk)), canon(ref.reshape(-1, wl.topk)))
     assert ic.get_device_status() == 0
 
 
