@@ -218,6 +218,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // the index rows may come from the previous kernel of a layer loop, and the
+    // outputs or partials may still be read by it
+    griddep_sync();
     const int n_rounds = ceil_div(p.n_work, static_cast<int>(gridDim.x));
     // copies issued by the producers' first thread: Q loads and KV tiles armed (counts)
     uint32_t q_armed = 0, kv_armed = 0;
@@ -460,7 +463,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         const int hb = Cfg::SMX_HEADS * sw;    // its heads: [hb, hb + 32)
         const int wtid = threadIdx.x - 128 * sw;
         const int sbar = 1 + sw;               // its named barrier
-        uint32_t t_it = 0, pv_it = 0;
+        uint32_t t_it = 0;  // tiles (and so P.V products) handled so far
         for (int r = 0; r < n_rounds; ++r) {
             const int item = attn_snake(r, blockIdx.x, gridDim.x);
             if (item >= p.n_work) continue;
@@ -508,13 +511,6 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                     zmax = fmaxf(zmax, valid ? z : -INFINITY);
                     sv[r2] = __float_as_uint(z);
                 }
-                // the previous tile's P.V must be complete before this tile's
-                // P is handed over (keeps the pv_done phase count in step and
-                // makes the accumulator safe to rescale)
-                if (j >= 1) {
-                    mbar_wait(bar_pv_done, pv_it & 1, abort_flag);
-                    ++pv_it;
-                }
                 if (named_bar_or(sbar, 128, zmax > IC_ATTN_RESCALE_LOG2)) {
                     // rare path: raise the reference to the tile maximum and
                     // rescale the accumulated output and row sums
@@ -549,6 +545,12 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                         sv[r2] = __float_as_uint(__uint_as_float(sv[r2]) - dz);
                     }
                     if (j >= 1) {
+                        // the previous tile's P.V must be complete before the
+                        // accumulator is rescaled. P.V(j-2) was issued before
+                        // QK(j) and the MMAs complete in issue order, so with S(j)
+                        // in hand the barrier is at most one phase behind P.V(j-1):
+                        // the parity wait is exact (P.V count = tile count)
+                        mbar_wait(bar_pv_done, (t_it - 1) & 1, abort_flag);
                         tc_fence_after();
                         for (int vb = 0; vb < Cfg::NVB; ++vb) {
                             {
@@ -603,10 +605,13 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 ++t_it;
             }
 
-            // ---- end of row: row sums, then the output (or the partials)
+            // ---- end of row: row sums, then the output (or the partials), once
+            // the row's last two P.V are complete (P.V(n-3) was issued before
+            // QK(n-1), so the barrier is at most two phases behind: wait for
+            // the second-to-last, then the last, each an exact parity wait)
             if (n_tiles > 0) {
-                mbar_wait(bar_pv_done, pv_it & 1, abort_flag);
-                ++pv_it;
+                if (n_tiles >= 2) mbar_wait(bar_pv_done, (t_it - 2) & 1, abort_flag);
+                mbar_wait(bar_pv_done, (t_it - 1) & 1, abort_flag);
                 tc_fence_after();
             }
 #pragma unroll
@@ -709,6 +714,7 @@ __global__ void __launch_bounds__(128)
                         int n_splits, int H, __nv_bfloat16* __restrict__ out) {
     // one CTA per (row, head); every thread derives the split weights itself
     // from the per-split running maximum m (log2 units) and sum l
+    griddep_sync();  // the partials come from the previous kernel
     const int64_t row = blockIdx.x / H;
     const int h = blockIdx.x % H;
     float m_c[8], w_c[8];

@@ -145,6 +145,24 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity,
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch. A kernel of the layer loop may be launched
+// while its predecessor (another kernel of this library) is still finishing.
+// Before a thread reads anything an earlier kernel of the loop wrote, or
+// writes any global memory, it waits for the predecessor grid to complete
+// (griddep_wait; a no-op for a kernel launched without the dependency). Only
+// then does the CTA allow its own dependents to launch, so a dependent can
+// never start while a kernel two launches back is still running.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_sync() {
+    griddep_wait();
+    griddep_launch_dependents();
+}
+
+// ---------------------------------------------------------------------------
 // Named barriers (a warpgroup synchronising among itself)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {

@@ -89,6 +89,26 @@ DeviceInfo device_info() {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Launch with an optional programmatic dependency on the previous kernel in
+// the stream (it may still be finishing when this one starts; the kernels
+// wait with griddep_wait before touching what it wrote). Only used when that
+// previous kernel is one of this library's: a caller's kernel may write what
+// a kernel reads before its wait.
+cudaError_t launch(const void* kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, void** args,
+                   bool pdl) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelExC(&cfg, kernel, args);
+}
 bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
 
 // A kernel that rebalances registers with setmaxnreg must have been launched
@@ -240,7 +260,7 @@ ic_status validate_indexer(const void* q_I, const float* q_scale, const void* w,
 ic_status launch_indexer(const void* q_I, const float* q_scale, const void* w, ic_dtype w_dt, const void* k_I,
                          const float* k_scale, ic_dtype qk_dt, int batch, int n_q, int n_k, int q_pos0, int H_I,
                          int d_I, int topk, int32_t* idx_out, void* ws, size_t ws_bytes, cudaStream_t stream,
-                         bool allow_dense = true) {
+                         bool allow_dense = true, bool pdl = false) {
     ic_status st = validate_indexer(q_I, q_scale, w, w_dt, k_I, k_scale, qk_dt, batch, n_q, n_k, q_pos0, H_I,
                                     d_I, topk, idx_out);
     if (st != IC_OK) return st;
@@ -285,15 +305,17 @@ ic_status launch_indexer(const void* q_I, const float* q_scale, const void* w, i
         if (e != cudaSuccess) return cuda_fail("decode indexer smem attribute", e);
         const int grid = std::max(1, std::min(d.n_work, dev.sms));
         void* args[] = {&tm_q, &tm_k, &d};
-        e = cudaLaunchKernel(pl.dec_kernel, dim3(grid), dim3(pl.dec_threads), args, pl.dec_smem, stream);
+        e = launch(pl.dec_kernel, dim3(grid), dim3(pl.dec_threads), pl.dec_smem, stream, args, pdl);
         if (e != cudaSuccess) return cuda_fail("decode indexer launch", e);
         const int rows_smem = ic::TOPK_ROWS_SMEM;
         e = cudaFuncSetAttribute(&ic::topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  ic::TOPK_ROWS_SMEM);
         if (e != cudaSuccess) return cuda_fail("top-k rows smem attribute", e);
-        ic::topk_rows_kernel<<<batch, ic::TOPK_ROWS_NT, rows_smem, stream>>>(d.scores, d.stride, d.n_vis, topk,
-                                                                             idx_out);
-        e = cudaGetLastError();
+        const uint32_t* sc_ptr = d.scores;
+        int stride = d.stride, n_vis = d.n_vis, kk = topk;
+        void* rargs[] = {&sc_ptr, &stride, &n_vis, &kk, &idx_out};
+        e = launch(reinterpret_cast<const void*>(&ic::topk_rows_kernel), dim3(batch), dim3(ic::TOPK_ROWS_NT),
+                   rows_smem, stream, rargs, true);
         if (e != cudaSuccess) return cuda_fail("top-k rows launch", e);
         return IC_OK;
     }
@@ -328,16 +350,20 @@ ic_status launch_indexer(const void* q_I, const float* q_scale, const void* w, i
     if (per_sm < 1) return cuda_fail("indexer occupancy", cudaErrorInvalidConfiguration);
     const int grid = std::max(1, std::min(p.n_work, dev.sms * per_sm));
     void* args[] = {&tm_q, &tm_k, &p};
-    e = cudaLaunchKernel(pl.kernel, dim3(grid), dim3(pl.threads), args, pl.smem, stream);
+    e = launch(pl.kernel, dim3(grid), dim3(pl.threads), pl.smem, stream, args, pdl);
     if (e != cudaSuccess) return cuda_fail("indexer launch", e);
     if (L.splits > 1) {
         constexpr int merge_smem = MERGE_MAX * 8;
         e = cudaFuncSetAttribute(&ic::topk_merge_kernel<MERGE_E>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  merge_smem);
         if (e != cudaSuccess) return cuda_fail("top-k merge smem attribute", e);
-        ic::topk_merge_kernel<MERGE_E><<<batch * n_q, 256, merge_smem, stream>>>(p.cand_key, p.cand_idx, p.cand_cnt,
-                                                                               L.splits, topk, idx_out);
-        e = cudaGetLastError();
+        const uint32_t* ckp = p.cand_key;
+        const int32_t* cip = p.cand_idx;
+        const int32_t* ccp = p.cand_cnt;
+        int splits = L.splits, kk = topk;
+        void* margs[] = {&ckp, &cip, &ccp, &splits, &kk, &idx_out};
+        e = launch(reinterpret_cast<const void*>(&ic::topk_merge_kernel<MERGE_E>), dim3(batch * n_q), dim3(256),
+                   merge_smem, stream, margs, true);
         if (e != cudaSuccess) return cuda_fail("top-k merge launch", e);
     }
     return IC_OK;
@@ -379,9 +405,13 @@ bool choose_attn_plan(int d_qk, int d_v, AttnPlan* pl) {
     return false;
 }
 
+#ifndef IC_ATTN_SPLIT_WAVES
+#define IC_ATTN_SPLIT_WAVES 1
+#endif
+
 int attn_splits(int rows, int topk, int sms) {
     if (rows <= 0 || sms <= 0 || rows >= sms) return 1;
-    int s = sms / rows;  // one round of work items: no CTA takes two
+    int s = IC_ATTN_SPLIT_WAVES * sms / rows;  // rounds of work items per CTA
     s = std::min(s, std::max(1, ceil_div(topk, 256)));
     s = std::min(s, 8);
     return std::max(s, 1);
@@ -395,7 +425,7 @@ size_t attn_ws_bytes(int rows, int splits, int H, int d_v) {
 
 ic_status launch_attn(const void* q, const void* kv, const int32_t* idx, int batch, int n_q, int n_k, int H, int d_qk,
                       int d_v, int topk, float sm_scale, void* out, void* ws, size_t ws_bytes,
-                      cudaStream_t stream) {
+                      cudaStream_t stream, bool pdl = false) {
     if (batch < 0 || n_q < 0 || n_k < 0 || H <= 0 || d_qk <= 0 || d_v <= 0 || topk <= 0) return IC_ERR_INVALID_ARG;
     if (batch == 0 || n_q == 0) return IC_OK;
     if (!q || !idx || !out || (n_k > 0 && !kv)) return IC_ERR_INVALID_ARG;
@@ -443,12 +473,12 @@ ic_status launch_attn(const void* q, const void* kv, const int32_t* idx, int bat
     if (e != cudaSuccess) return cuda_fail("attention smem attribute", e);
     const int grid = std::max(1, std::min(p.n_work, dev.sms));
     void* args[] = {&tm_q, &tm_kv, &p};
-    e = cudaLaunchKernel(pl.kernel, dim3(grid), dim3(pl.threads), args, pl.smem, stream);
+    e = launch(pl.kernel, dim3(grid), dim3(pl.threads), pl.smem, stream, args, pdl);
     if (e != cudaSuccess) return cuda_fail("attention launch", e);
     if (splits > 1) {
         int sp = splits, hh = H;
         void* cargs[] = {&p.o_part, &p.ml_part, &sp, &hh, &p.out};
-        e = cudaLaunchKernel(reinterpret_cast<const void*>(pl.combine), dim3(rows * H), dim3(128), cargs, 0, stream);
+        e = launch(reinterpret_cast<const void*>(pl.combine), dim3(rows * H), dim3(128), 0, stream, cargs, true);
         if (e != cudaSuccess) return cuda_fail("attention combine launch", e);
     }
     return IC_OK;
@@ -793,17 +823,22 @@ ic_status ic_layer_stack(const ic_layer_io* layers, int n_layers, int index_topk
         if (s->batch > 0 && s->n_q > 0 && (!L.q || !L.out || (s->n_k > 0 && !L.kv))) return IC_ERR_INVALID_ARG;
     }
     const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    // every launch after the call's first follows one of this library's
+    // kernels: it may start while that one finishes (programmatic dependency)
+    bool pdl = false;
     for (int l = 0; l < n_layers; ++l) {
         const ic_layer_io& L = layers[l];
         if (is_full[l]) {  // the single conditional branch: Full layers refresh the cached indices
             st = launch_indexer(L.q_I, L.q_scale, L.w, s->w_dtype, L.k_I, L.k_scale, s->qk_dtype, s->batch, s->n_q,
                                 s->n_k, s->q_pos0, s->H_I, s->d_I, s->topk, idx_buffer, workspace, workspace_bytes,
-                                cs);
+                                cs, true, pdl);
             if (st != IC_OK) return st;
+            pdl = true;
         }
         st = launch_attn(L.q, L.kv, idx_buffer, s->batch, s->n_q, s->n_k, s->H, s->d_qk, s->d_v, s->topk, s->sm_scale,
-                         L.out, workspace, workspace_bytes, cs);
+                         L.out, workspace, workspace_bytes, cs, pdl);
         if (st != IC_OK) return st;
+        pdl = true;
     }
     return IC_OK;
 }

@@ -345,7 +345,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
             const IdxWork wk = idx_work<Cfg>(p, item);
             const int c_split = item % p.n_splits;
             if (wk.trivial) {
-                // every visible key is selected: 0..n_vis-1, then -1
+                // every visible key is selected: 0..n_vis-1, then -1 (the index
+                // buffer may still be read by the previous kernel of a layer loop)
+                griddep_sync();
                 for (int gl = 0; gl < QPW; ++gl) {
                     const int g = e * QPW + gl;
                     if (g >= wk.nq_valid) continue;
@@ -482,7 +484,6 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_acc_empty(a));
                 const bool meet = (t + 1) % per == 0 && t + 1 < wk.n_tiles;  // same in every epilogue thread
-                if (!meet && t + 1 < wk.n_tiles) issue_loads(ait + 1);
                 float pk[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
@@ -521,6 +522,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                     }
                 }
 
+                // the next tile's TMEM loads go out after the append (issued before
+                // it, they measured ~500 cycles per tile slower)
+                if (!meet && t + 1 < wk.n_tiles) issue_loads(ait + 1);
                 if (meet) {
                     // ---- meeting: every list's appends so far are done; the OR says
                     // whether any list passed hw
@@ -554,7 +558,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                     issue_loads(ait + 1);
                 }
               }
-              // every warp's appends must be visible to the final select
+              // every warp's appends must be visible to the final select; the
+              // outputs may still be read by the previous kernel of a layer loop
+              griddep_sync();
               named_bar_sync(bar_id, 128);
               if (e < wk.nq_valid) {  // uniform across the warpgroup
                   const int n = static_cast<int>(st.fcount);
@@ -760,7 +766,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
               }
               par ^= 1;
             }
-            // candidates appended by the other warps must be visible to the final select
+            // candidates appended by the other warps must be visible to the final
+            // select; the outputs may still be read by the previous kernel
+            griddep_sync();
             named_bar_sync(bar_id, 128);
 
             // ---- final exact selection for each query of this warpgroup
@@ -842,6 +850,7 @@ __global__ void __launch_bounds__(256)
     int32_t* midx = reinterpret_cast<int32_t*>(merge_smem + 256 * E);
     const int row = blockIdx.x;
     const int tid = threadIdx.x;
+    griddep_sync();  // the candidate lists come from the previous kernel
     if (tid == 0) {
         int o = 0;
         for (int c = 0; c < n_splits; ++c) {

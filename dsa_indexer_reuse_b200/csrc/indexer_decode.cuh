@@ -234,6 +234,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     } else {
         regs_inc<Cfg::REGS_EPI>();
         // ------------------------------------------------------------ epilogue
+        // the score rows go to the caller's workspace, which the previous
+        // kernel of a layer loop may still be using
+        griddep_sync();
         const int e = (warp - 4) >> 2;  // warpgroup: tiles with seq % 4 == e
         const int wq = warp & 3;        // TMEM lane quarter
         const int c4 = lane & 3, r8 = lane >> 2;
@@ -354,6 +357,7 @@ __global__ void __launch_bounds__(TOPK_ROWS_NT)
     int32_t* pidx = reinterpret_cast<int32_t*>(pkey + TOPK_ROWS_PRE);
     const int row = blockIdx.x;
     const int tid = threadIdx.x;
+    griddep_sync();  // the score rows come from the previous kernel
     // stride is a multiple of 128 keys, so every row starts 16-byte aligned
     const uint4* src = reinterpret_cast<const uint4*>(scores + static_cast<int64_t>(row) * stride);
     for (int i = tid; i < (n_vis + 3) / 4; i += TOPK_ROWS_NT) rows_smem[i] = __ldg(src + i);

@@ -522,10 +522,11 @@ template <int NT, int E, class Keep, class Group, class Emit>
 __device__ int comp_emit_grouped(int n, int tid, int bar_id, CompScratch<NT, E>& sc, Keep&& keep, Group&& group,
                                  Emit&& emit) {
     constexpr int NW = NT / 32;
-    constexpr int NG = CompScratch<NT, E>::NG;
     constexpr int NTB = CompScratch<NT, E>::NTBL;
     const int lane = tid & 31, warp = tid >> 5;
-    uint32_t kmask = 0, gbits0 = 0, gbits1 = 0;  // group of round m: bit m of gbits0 | 2 * bit m of gbits1
+    // bin of round m: its group (0..3), or -1 when the position is not kept;
+    // two bits per round (group + 1 in 0..4 needs three: kept mask apart)
+    uint32_t kmask = 0, gbits0 = 0, gbits1 = 0;
 #pragma unroll 8
     for (int m = 0; m < E; ++m) {
         const int pos = m * NT + tid;
@@ -536,20 +537,17 @@ __device__ int comp_emit_grouped(int n, int tid, int bar_id, CompScratch<NT, E>&
             gbits1 |= static_cast<uint32_t>((g >> 1) & 1) << m;
         }
     }
-    auto grp = [&](int m) { return static_cast<int>(((gbits0 >> m) & 1u) | (((gbits1 >> m) & 1u) << 1)); };
-    int cnt[NG] = {0, 0, 0, 0};
+    auto bin_of = [&](int m) {
+        return ((kmask >> m) & 1u) ? static_cast<int>(((gbits0 >> m) & 1u) | (((gbits1 >> m) & 1u) << 1)) : -1;
+    };
+    for (int i = tid; i < NTB; i += NT) sc.tbl[i] = 0;
+    named_bar_sync(bar_id, NT);
+    // per (group, round, warp): the lowest lane of each group writes its count
 #pragma unroll
     for (int m = 0; m < E; ++m) {
-        const bool kp = (kmask >> m) & 1u;
-#pragma unroll
-        for (int g = 0; g < NG; ++g) {
-            const uint32_t b = __ballot_sync(0xffffffffu, kp && grp(m) == g);
-            if (lane == m) cnt[g] = __popc(b);
-        }
-    }
-    if (lane < E) {
-#pragma unroll
-        for (int g = 0; g < NG; ++g) sc.tbl[(g * E + lane) * NW + warp] = cnt[g];
+        const int b = bin_of(m);
+        const uint32_t peers = __match_any_sync(0xffffffffu, b);
+        if (b >= 0 && lane == __ffs(peers) - 1) sc.tbl[(b * E + m) * NW + warp] = __popc(peers);
     }
     named_bar_sync(bar_id, NT);
     // exclusive scan over the (group, round, warp) table: each thread scans a
@@ -565,7 +563,6 @@ __device__ int comp_emit_grouped(int n, int tid, int bar_id, CompScratch<NT, E>&
     }
     int ex, ex_b, tot, tot_b;
     block_scan2<NT>(run_sum, 0, ex, ex_b, tot, tot_b, sc.scan_tmp, tid, bar_id);
-    named_bar_sync(bar_id, NT);  // every thread has read its run
 #pragma unroll
     for (int i = 0; i < RUN; ++i) {
         const int e = tid * RUN + i;
@@ -576,13 +573,9 @@ __device__ int comp_emit_grouped(int n, int tid, int bar_id, CompScratch<NT, E>&
     const uint32_t lt = lanemask_lt();
 #pragma unroll 4
     for (int m = 0; m < E; ++m) {
-        const bool kp = (kmask >> m) & 1u;
-        const int gm = grp(m);
-#pragma unroll
-        for (int g = 0; g < NG; ++g) {
-            const uint32_t b = __ballot_sync(0xffffffffu, kp && gm == g);
-            if (kp && gm == g) emit(sc.tbl[(g * E + m) * NW + warp] + __popc(b & lt), m * NT + tid);
-        }
+        const int b = bin_of(m);
+        const uint32_t peers = __match_any_sync(0xffffffffu, b);
+        if (b >= 0) emit(sc.tbl[(b * E + m) * NW + warp] + __popc(peers & lt), m * NT + tid);
     }
     named_bar_sync(bar_id, NT);  // the table may be reused
     return tot;
