@@ -96,6 +96,15 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                  : "memory");
 }
 
+// First 1024-byte aligned byte of dynamic shared memory. The offset is
+// taken from the shared-window address and applied to the shared pointer
+// itself, so accesses through the result stay shared-memory instructions
+// (a round trip through an integer would make them generic).
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* smem_raw) {
+    const uint32_t a = smem_u32(smem_raw);
+    return smem_raw + (((a + 1023u) & ~1023u) - a);
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(

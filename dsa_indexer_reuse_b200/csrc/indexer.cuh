@@ -190,8 +190,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                         const __grid_constant__ CUtensorMap tm_k, const IdxParams p) {
     constexpr int HI = Cfg::HI, G = Cfg::G, QPW = Cfg::QPW, E = Cfg::E, C = Cfg::C;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* smem = align_smem_1024(smem_raw);
     const uint32_t s_base = smem_u32(smem);
     uint32_t* cand_key_s = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_CK);
     int32_t* cand_idx_s = reinterpret_cast<int32_t*>(smem + Cfg::OFF_CI);
@@ -428,20 +427,28 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
               // warp's lane quarter, 16 heads each. The loads of tile t+1 are
               // issued before the append of tile t, so their latency overlaps it.
               uint32_t ra[32], rb[32];
+              const uint32_t tb0 = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + e * Cfg::COLS_PER_WG;
               auto issue_loads = [&](uint32_t it) {
                   mbar_wait(bar_acc_full(it & 1), (it >> 1) & 1, abort_flag);
                   tc_fence_after();
-                  const uint32_t tb = tmem_base + (static_cast<uint32_t>(wq * 32) << 16) + (it & 1) * Cfg::N +
-                                      e * Cfg::COLS_PER_WG;
+                  const uint32_t tb = tb0 + (it & 1) * Cfg::N;
                   tmem_ld_16x256b_x8(tb, ra);
                   tmem_ld_16x256b_x8(tb + (16u << 16), rb);
               };
+              // per-item constants of the tile loop: the last key this lane's
+              // query may select (-1: none), the key scales of the batch element
+              const int key_hi = e < wk.nq_valid ? min(wk.k_end - 1, pos_g) : -1;
+              const float* ks_row = p.k_scale != nullptr ? p.k_scale + static_cast<int64_t>(wk.b) * p.n_k : nullptr;
+              auto scale_of = [&](int sk) { return (ks_row != nullptr && sk < wk.k_end) ? ks_row[sk] : 1.f; };
+              int s_key = wk.k_begin + key_lane;  // this lane's key in the current tile
+              float ksc_f = scale_of(s_key);
+              int till_meet = per;
               if (wk.n_tiles > 0) issue_loads(ait);
-              for (int t = 0; t < wk.n_tiles; ++t, ++ait) {
+              for (int t = 0; t < wk.n_tiles; ++t, ++ait, s_key += IDX_BM) {
                 const int a = ait & 1;
                 // the next tile's key scale is requested a whole tile ahead
-                const float ksc = ksc_next;
-                ksc_next = key_scale(t + 1);
+                const float ksc = ksc_f;
+                ksc_f = scale_of(s_key + IDX_BM);
                 // this lane's 16 head weights (8-byte loads shared by the 8 lanes
                 // of a column pair)
                 float2 wreg[8];
@@ -483,7 +490,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_acc_empty(a));
-                const bool meet = (t + 1) % per == 0 && t + 1 < wk.n_tiles;  // same in every epilogue thread
+                // every `per` tiles, except after the last: the same in every epilogue thread
+                const bool meet = --till_meet == 0 && t + 1 < wk.n_tiles;
+                if (till_meet == 0) till_meet = per;
                 float pk[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
@@ -499,8 +508,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 const bool hi2 = (c4 & 2) != 0;
                 const float sum = (hi2 ? q1 : q0) + __shfl_xor_sync(0xffffffffu, hi2 ? q0 : q1, 2);
                 const uint32_t kk = float_to_ordered(sum * ksc);
-                const int s_key = wk.k_begin + t * IDX_BM + key_lane;
-                const bool valid = s_key < wk.k_end && e < wk.nq_valid && s_key <= pos_g;
+                const bool valid = s_key <= key_hi;
 
                 // ---- append this tile's passing keys (one atomic per warp)
                 const bool pass = valid && comp_key(kk, s_key) > thr;

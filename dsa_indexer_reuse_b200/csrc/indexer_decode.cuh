@@ -97,8 +97,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                                  const IdxDecParams p) {
     constexpr int HI = Cfg::HI;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* smem = align_smem_1024(smem_raw);
     const uint32_t s_base = smem_u32(smem);
     const uint32_t bar0 = s_base + Cfg::OFF_BAR;
     auto bar_k_full = [&](int s) { return bar0 + 8u * s; };

@@ -542,12 +542,17 @@ __device__ int comp_emit_grouped(int n, int tid, int bar_id, CompScratch<NT, E>&
     };
     for (int i = tid; i < NTB; i += NT) sc.tbl[i] = 0;
     named_bar_sync(bar_id, NT);
-    // per (group, round, warp): the lowest lane of each group writes its count
+    // per (group, round, warp): one ballot per group; lane g writes group g's count
 #pragma unroll
     for (int m = 0; m < E; ++m) {
         const int b = bin_of(m);
-        const uint32_t peers = __match_any_sync(0xffffffffu, b);
-        if (b >= 0 && lane == __ffs(peers) - 1) sc.tbl[(b * E + m) * NW + warp] = __popc(peers);
+        int mine = 0;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const int c = __popc(__ballot_sync(0xffffffffu, b == g));
+            if (lane == g) mine = c;
+        }
+        if (lane < 4) sc.tbl[(lane * E + m) * NW + warp] = mine;
     }
     named_bar_sync(bar_id, NT);
     // exclusive scan over the (group, round, warp) table: each thread scans a
@@ -574,7 +579,12 @@ __device__ int comp_emit_grouped(int n, int tid, int bar_id, CompScratch<NT, E>&
 #pragma unroll 4
     for (int m = 0; m < E; ++m) {
         const int b = bin_of(m);
-        const uint32_t peers = __match_any_sync(0xffffffffu, b);
+        uint32_t peers = 0;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const uint32_t bg = __ballot_sync(0xffffffffu, b == g);
+            if (b == g) peers = bg;
+        }
         if (b >= 0) emit(sc.tbl[(b * E + m) * NW + warp] + __popc(peers & lt), m * NT + tid);
     }
     named_bar_sync(bar_id, NT);  // the table may be reused
