@@ -117,6 +117,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Like mbar_try_wait, but a thread whose phase is not complete may be
+// suspended until it completes or for at most IC_WAIT_SUSPEND_NS: the waiting
+// loops below poll far less often (fewer issue slots taken from the warps
+// that share the scheduler).
+#ifndef IC_WAIT_SUSPEND_NS
+#define IC_WAIT_SUSPEND_NS 1000000u  // 1 ms
+#endif
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(static_cast<uint32_t>(IC_WAIT_SUSPEND_NS))
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity to complete. Returns
 // false (without waiting) once the CTA is in abort mode, or after the
 // timeout, which also puts the CTA in abort mode.
@@ -127,7 +146,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     const uint64_t t0 = globaltimer_ns();
     uint32_t spins = 0;
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_suspend(bar, parity)) return true;
         if ((++spins & 15u) == 0) {
             if (*abort_flag) return false;
             if (globaltimer_ns() - t0 > timeout_ns) {
@@ -145,7 +164,7 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity,
                                            uint64_t timeout_ns = IC_WAIT_TIMEOUT_NS) {
     if (mbar_try_wait(bar, parity)) return;
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_suspend(bar, parity)) {
         if (globaltimer_ns() - t0 > timeout_ns) {
             record_status(IC_ERR_TIMEOUT);
             return;

@@ -248,6 +248,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             uint32_t kst = 0, qit = 0;
+            int ks_stage = 0;        // kst % STAGES
+            uint32_t ks_phase = 0;   // (kst / STAGES) & 1
             for (int r = 0; r < n_rounds; ++r) {
                 const int item = snake_item(r, blockIdx.x, gridDim.x);
                 if (item >= p.n_work) continue;
@@ -265,8 +267,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 }
                 ++qit;
                 for (int t = 0; t < wk.n_tiles; ++t) {
-                    const int s = kst % Cfg::STAGES;
-                    if (mbar_wait(bar_empty(s), ((kst / Cfg::STAGES) & 1) ^ 1, abort_flag)) {
+                    const int s = ks_stage;
+                    if (mbar_wait(bar_empty(s), ks_phase ^ 1, abort_flag)) {
                         mbar_arrive_expect_tx(bar_full(s), Cfg::K_BYTES);
                         const int krow = wk.b * p.n_k + wk.k_begin + t * IDX_BM;
 #pragma unroll
@@ -276,13 +278,19 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                         k_armed = kst + 1;
                     }
                     ++kst;
+                    if (++ks_stage == Cfg::STAGES) {
+                        ks_stage = 0;
+                        ks_phase ^= 1;
+                    }
                 }
             }
         }
       } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            uint32_t kst = 0, qit = 0, ait = 0;
+            uint32_t qit = 0, ait = 0;
+            int ks_stage = 0;        // key tile count % STAGES
+            uint32_t ks_phase = 0;   // (key tile count / STAGES) & 1
             for (int r = 0; r < n_rounds; ++r) {
                 const int item = snake_item(r, blockIdx.x, gridDim.x);
                 if (item >= p.n_work) continue;
@@ -292,13 +300,17 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 ++qit;
                 tc_fence_after();
                 for (int t = 0; t < wk.n_tiles; ++t) {
-                    const int s = kst % Cfg::STAGES;
+                    const int s = ks_stage;
+                    const uint32_t kph = ks_phase;
+                    if (++ks_stage == Cfg::STAGES) {
+                        ks_stage = 0;
+                        ks_phase ^= 1;
+                    }
                     const int a = ait & 1;
-                    const bool go = mbar_wait(bar_full(s), (kst / Cfg::STAGES) & 1, abort_flag) &&
+                    const bool go = mbar_wait(bar_full(s), kph, abort_flag) &&
                                     mbar_wait(bar_acc_empty(a), ((ait >> 1) & 1) ^ 1, abort_flag);
                     tc_fence_after();
                     if (!go) {  // aborted: issue nothing more; the teardown drains
-                        ++kst;
                         ++ait;
                         continue;
                     }
@@ -318,7 +330,6 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                     }
                     mma_commit(bar_empty(s));
                     mma_commit(bar_acc_full(a));
-                    ++kst;
                     ++ait;
                 }
                 mma_commit(bar_q_empty);
