@@ -44,6 +44,7 @@ struct DistillParams {
     int fp8;
     const int32_t* idx;     // [batch * n_q, topk]
     int n_q, n_k, topk, H, d_I;
+    int rows;               // batch * n_q
     float sm_scale;
     float* target;          // [batch * n_q, topk] or null
     float* kl;              // [batch * n_q]

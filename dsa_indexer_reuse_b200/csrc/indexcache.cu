@@ -25,6 +25,7 @@
 #include "indexer.cuh"
 #include "indexer_decode.cuh"
 #include "distill.cuh"
+#include "distill_tc.cuh"
 #include "overlap.cuh"
 
 namespace {
@@ -541,6 +542,22 @@ ic_status launch_distill(const ic::DistillParams& p, int rows, cudaStream_t stre
     ic::distill_target_kernel<DQK, HI><<<rows, ic::DISTILL_THREADS, smem, stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("distill launch", e);
+    return IC_OK;
+}
+
+template <class Cfg>
+ic_status launch_distill_tc(const ic::DistillParams& p, cudaStream_t stream) {
+    cudaError_t e = cudaFuncSetAttribute(ic::distill_tc_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg::SMEM_ALLOC);
+    if (e != cudaSuccess) return cuda_fail("distill (tensor cores) smem attribute", e);
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return cuda_fail("SM count", e);
+    const int grid = std::max(1, std::min(p.rows, sms));
+    ic::distill_tc_kernel<Cfg><<<grid, Cfg::THREADS, Cfg::SMEM_ALLOC, stream>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("distill (tensor cores) launch", e);
     return IC_OK;
 }
 
@@ -1171,7 +1188,13 @@ ic_status ic_distill_target(const void* const* q_layers, const void* const* kv_l
     p.target = target_out;
     p.kl = kl_out;
     const int rows = batch * n_q;
+    p.rows = rows;
     const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    // the model's shapes (64 heads over 576-wide latent rows, a 64-head
+    // 128-wide indexer) run on the tensor cores; other shapes on the CUDA cores
+    if (H == 64 && d_qk == 576 && H_I == 64 && d_I == 128 && aligned16(q_I))
+        return p.fp8 ? launch_distill_tc<ic::DistTcCfg<576, true>>(p, cs)
+                     : launch_distill_tc<ic::DistTcCfg<576, false>>(p, cs);
     if (d_qk == 576) return H_I == 64 ? launch_distill<576, 64>(p, rows, cs) : launch_distill<576, 4>(p, rows, cs);
     return H_I == 64 ? launch_distill<64, 64>(p, rows, cs) : launch_distill<64, 4>(p, rows, cs);
 }

@@ -96,3 +96,26 @@ def test_unsupported_shapes_are_refused(cuda_ok):
     with pytest.raises(ic.IcError) as e:
         ic.distill_target(served * 65, ind["q_I"], ind["w"], ind["k_I"], idx)
     assert e.value.code == 3  # IC_ERR_UNSUPPORTED
+
+
+def test_latent_rows_without_keys_and_out_of_range_entries(cuda_ok):
+    # the tensor-core configuration (64 heads, 576-wide rows, 64-head indexer)
+    wl = W.PREFILL_8K.with_(n_q=192, n_k=192, topk=128, n_layers=2)
+    ind, served, idx = _inputs(wl, 2, seed=10)
+    idx = idx.clone()
+    idx[0, 5] = -1            # no valid entry
+    idx[0, 9, :7] = 4096      # out of range: skipped
+    idx[0, 150, ::3] = -1     # holes inside a row
+    t, kl = _check(wl, ind, served, idx)
+    assert kl[5] == 0.0 and (t[5] == 0).all()
+    assert (t[9, :7] == 0).all() and (t[150, ::3] == 0).all()
+
+
+def test_latent_long_rows_peaked_logits(cuda_ok):
+    # rows of 1536 keys (12 tiles of 128: the first 4 are computed twice) and
+    # logits with a standard deviation of ~32, so every head's softmax is
+    # dominated by a few keys and the running maxima matter
+    wl = W.DECODE_32X32K.with_(batch=2, n_k=1536, q_pos0=1535, n_layers=2)
+    ind, served, idx = _inputs(wl, 2, seed=12)
+    served = [(q * 32, kv) for q, kv in served]
+    _check(wl, ind, served, idx)
