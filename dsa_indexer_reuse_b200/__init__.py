@@ -16,7 +16,8 @@ Entry points (same names as the C ABI, without the ``ic_`` prefix):
     topk_overlap, search_pattern, greedy_pattern (pattern tools), and
     overlap_matrix (layer x layer ratios), pattern_score (the search
     objective of one pattern), and
-    distill_target (the multi-layer distillation target and KL of one Full layer).
+    distill_target (the multi-layer distillation target and KL of one Full layer)
+    with distill_target_workspace_size.
 The submodule ``workloads`` (seeded synthetic inputs) needs no library.
 """
 
@@ -26,6 +27,7 @@ _EXPORTS = (
     "layer_stack_workspace_size", "lib", "resolve_pattern", "sparse_attn",
     "sparse_attn_workspace_size", "version", "topk_overlap", "overlap_matrix", "search_pattern",
     "greedy_pattern", "pattern_score", "StackHostCall", "layer_stack_host", "distill_target",
+    "distill_target_workspace_size",
 )
 
 

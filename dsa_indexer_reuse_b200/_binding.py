@@ -85,8 +85,10 @@ lib.ic_layer_stack_host.argtypes = [ctypes.POINTER(_LayerIO), _I, _I, ctypes.c_c
                                     ctypes.POINTER(_StackShape), _P, _P, _SZ, _P,
                                     ctypes.POINTER(_SZ), ctypes.POINTER(_SZ)]
 lib.ic_layer_stack_host.restype = _I
+lib.ic_distill_target_workspace_size.argtypes = [_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)]
+lib.ic_distill_target_workspace_size.restype = _I
 lib.ic_distill_target.argtypes = [_P, _P, _I, _P, _P, _P, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I,
-                                  _I, _I, ctypes.c_float, _P, _P, _P]
+                                  _I, _I, ctypes.c_float, _P, _P, _P, _SZ, _P]
 lib.ic_distill_target.restype = _I
 lib.ic_get_device_status.argtypes = [_I]
 lib.ic_get_device_status.restype = _I
@@ -339,8 +341,15 @@ def layer_stack_host(layers, shape: dict, *, freq=0, pattern=None, idx_out=None,
     return StackHostCall(layers, shape, freq=freq, pattern=pattern, idx_out=idx_out)(stream)
 
 
+def distill_target_workspace_size(batch, n_q, topk, H, d_qk, H_I, d_I) -> int:
+    out = _SZ(0)
+    _check(lib.ic_distill_target_workspace_size(batch, n_q, topk, H, d_qk, H_I, d_I, ctypes.byref(out)),
+           "ic_distill_target_workspace_size")
+    return int(out.value)
+
+
 def distill_target(served, q_I, w, k_I, idx, *, q_scale=None, k_scale=None, sm_scale=None,
-                   with_target=True, stream=None):
+                   with_target=True, workspace=None, stream=None):
     """Multi-layer distillation target of one Full layer (ic_distill_target).
     `served`: list of (q [B, n_q, H, d_qk], kv [B, n_k, d_qk]) bf16 tensors of
     the layers it serves (itself first, by convention); q_I, w, k_I (and the
@@ -360,10 +369,13 @@ def distill_target(served, q_I, w, k_I, idx, *, q_scale=None, k_scale=None, sm_s
     dev = idx.device
     target = torch.empty((B, n_q, topk), dtype=torch.float32, device=dev) if with_target else None
     kl = torch.empty((B, n_q), dtype=torch.float32, device=dev)
+    ws_bytes = distill_target_workspace_size(B, n_q, topk, H, d_qk, H_I, d_I)
+    workspace, ws_len = _workspace(ws_bytes, dev, workspace)
     code = lib.ic_distill_target(ctypes.cast(q_arr, ctypes.c_void_p), ctypes.cast(kv_arr, ctypes.c_void_p),
                                  len(served), _ptr(q_I), _ptr(q_scale), _ptr(w), _w_code(w), _ptr(k_I),
                                  _ptr(k_scale), _qk_code(q_I), _ptr(idx), B, n_q, n_k, H_I, d_I, topk, H,
-                                 d_qk, float(sm_scale), _ptr(target), _ptr(kl), _stream(stream))
+                                 d_qk, float(sm_scale), _ptr(target), _ptr(kl), _ptr(workspace), ws_len,
+                                 _stream(stream))
     _check(code, "ic_distill_target")
     return target, kl
 

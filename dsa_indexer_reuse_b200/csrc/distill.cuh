@@ -45,6 +45,7 @@ struct DistillParams {
     const int32_t* idx;     // [batch * n_q, topk]
     int n_q, n_k, topk, H, d_I;
     int rows;               // batch * n_q
+    void* spill;            // tensor-core kernel: per-CTA logit workspace
     float sm_scale;
     float* target;          // [batch * n_q, topk] or null
     float* kl;              // [batch * n_q]

@@ -19,11 +19,12 @@
 //    slots; the query rows stay resident, 128-byte swizzled, K-major.
 //  * Tensor memory holds eight 64-column accumulators. A head's softmax needs
 //    its normaliser over all keys before any probability is final, so every
-//    tile is read twice: a statistics pass (a running max and sum of
-//    exponentials per head and per thread, merged across the keys' threads
-//    at the end) and a probability pass. The last eight tiles of a row-layer
-//    stay in tensor memory between the two passes; earlier tiles are computed
-//    again for the probability pass (rows of at most 1024 keys: no recompute).
+//    tile's logits are read twice: a statistics pass (a running max and sum of
+//    exponentials per head and per thread, merged across the keys' threads at
+//    the end) and a probability pass. The last eight tiles of a row-layer stay
+//    in tensor memory between the two passes; the logits of earlier tiles (up
+//    to 8 x 32 KB per CTA) wait in a global workspace, which costs less than
+//    gathering and multiplying those tiles again.
 //  * The indexer scores of the same keys use the same machinery (K = 128:
 //    kind::f16 for bf16, kind::f8f6f4 for E4M3), followed by ReLU, the head
 //    weights and the scales in the epilogue; then the softmax of the scores
@@ -31,8 +32,9 @@
 //    the index row's positions (0 at invalid ones).
 //
 // Warp roles (512 threads): warps 0-3 epilogue (one thread per TMEM lane),
-// warp 4 MMA issuer and TMEM owner, warps 5-15 index compaction and the
-// cp.async gathers of query rows and key-row chunks.
+// warp 4 MMA issuer and TMEM owner, warps 5-12 the cp.async gathers of
+// key-row chunks, warps 13-15 the index compaction, the query-row loads and
+// L2 prefetches of the row's selected keys, one row ahead of the gathers.
 #pragma once
 
 #include "distill.cuh"
@@ -51,13 +53,20 @@ struct DistTcCfg {
     static constexpr int NCH = DQK / 64;           // 128-byte chunks of a latent row
     static constexpr int NCH_I = FP8I ? 1 : 2;     // 128-byte chunks of an indexer key row
     static constexpr int CH_BYTES = BM * 128;      // one ring slot: 128 rows x 128 B
-    static constexpr int NS = FP8I ? 6 : 5;        // ring slots
+    static constexpr int NS = 6;                   // ring slots
     static constexpr int NSLOT = 8;                // TMEM accumulators of 64 columns
     static constexpr int RESIDENT = NSLOT;         // tiles kept between the two passes
+    // logits of the other tiles of a row-layer (at most MAX_TOPK / BM - RESIDENT),
+    // fp32, per CTA: [tile][16 groups of 4 heads][128 keys] float4
+    static constexpr int SPILL_TILES = 2048 / BM - RESIDENT;
+    static constexpr size_t SPILL_BYTES_PER_CTA = static_cast<size_t>(SPILL_TILES) * BM * 64 * 4;
     static constexpr int MAX_TOPK = 2048;
     static constexpr int THREADS = 512;
     static constexpr int MMA_WARP = 4;
-    static constexpr int NPROD = 11 * 32;          // warps 5..15
+    static constexpr int AUX_WARP0 = 13;           // warps 5..12 gather key rows, 13..15 the rest
+    static constexpr int NGATHER = 32 * (AUX_WARP0 - MMA_WARP - 1);
+    static constexpr int NAUX = 32 * (16 - AUX_WARP0);
+    static_assert(NGATHER == 256, "four 16-byte units of every 128-row chunk per gather thread");
     static constexpr int REGS_EPI = 200, REGS_OTHER = 104;
     static_assert(128 * REGS_EPI + 384 * REGS_OTHER <= 65536, "register split");
     static constexpr uint32_t IDESC_S = make_idesc(BM, H, FMT_BF16, FMT_BF16);
@@ -89,17 +98,17 @@ struct DistTcCfg {
 // Number of tiles of a row of n valid keys.
 __device__ __forceinline__ int dist_tiles(int n) { return (n + 127) >> 7; }
 
-// Tiles computed a second time for the probability pass: those that did not
-// stay in tensor memory.
+// Tiles of a row-layer that do not stay in tensor memory between the two
+// passes: the first T - RESIDENT, whose logits wait in the spill workspace.
 template <class Cfg>
-__device__ __forceinline__ int dist_recompute(int T) {
+__device__ __forceinline__ int dist_spilled(int T) {
     return T > Cfg::RESIDENT ? T - Cfg::RESIDENT : 0;
 }
 
 template <class Cfg>
 __global__ void __launch_bounds__(Cfg::THREADS, 1) distill_tc_kernel(const __grid_constant__ DistillParams p) {
     constexpr int NS = Cfg::NS, NSLOT = Cfg::NSLOT, NCH = Cfg::NCH, NCH_I = Cfg::NCH_I;
-    constexpr int NPROD = Cfg::NPROD, MMA_WARP = Cfg::MMA_WARP, DQK = Cfg::DQK;
+    constexpr int MMA_WARP = Cfg::MMA_WARP, DQK = Cfg::DQK;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align_smem_1024(smem_raw);
     const uint32_t s_base = smem_u32(smem);
@@ -110,7 +119,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) distill_tc_kernel(const __gri
     float* hl_s = reinterpret_cast<float*>(smem + Cfg::OFF_HL);
     float* red_s = reinterpret_cast<float*>(smem + Cfg::OFF_RED);
     float* w_s = reinterpret_cast<float*>(smem + Cfg::OFF_W);
-    int* misc_s = reinterpret_cast<int*>(smem + Cfg::OFF_MISC);  // [0,2): n per list buffer; [8,19), [24,28): scans
+    int* misc_s = reinterpret_cast<int*>(smem + Cfg::OFF_MISC);  // [0,2): n per list buffer; [8,11), [24,28): scans
     const uint32_t bar0 = s_base + Cfg::OFF_BAR;
     auto bar_ring_full = [&](int s) { return bar0 + 8u * s; };
     auto bar_ring_empty = [&](int s) { return bar0 + 8u * (NS + s); };
@@ -128,16 +137,16 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) distill_tc_kernel(const __gri
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
-            mbar_init(bar_ring_full(s), NPROD);
+            mbar_init(bar_ring_full(s), Cfg::NGATHER);
             mbar_init(bar_ring_empty(s), 1);
         }
         for (int s = 0; s < NSLOT; ++s) {
             mbar_init(bar_acc_full(s), 1);
             mbar_init(bar_acc_empty(s), 4);
         }
-        mbar_init(bar_q_full, NPROD);
+        mbar_init(bar_q_full, Cfg::NAUX);
         mbar_init(bar_q_empty, 1);
-        mbar_init(bar_qi_full, NPROD);
+        mbar_init(bar_qi_full, Cfg::NAUX);
         mbar_init(bar_qi_empty, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_list_full(b), 1);
@@ -164,36 +173,71 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) distill_tc_kernel(const __gri
     if (warp >= 4) {
       regs_dec<Cfg::REGS_OTHER>();
       if (warp != MMA_WARP) {
-        // ------------------------------------------- compaction and gathers
-        const int ptid = threadIdx.x - 160;  // 0 .. NPROD-1
-        const int pw = ptid >> 5;
+        if (warp < Cfg::AUX_WARP0) {
+        // --------------------------------------------- key-row chunk gathers
+        // Thread gt copies 16-byte unit x = gt % 8 of rows gt / 8 + 32 k
+        // (k = 0..3) of every chunk: the same four rows for all chunks of a
+        // tile, so a tile's source rows are looked up once.
+        const int gt = threadIdx.x - 32 * (Cfg::MMA_WARP + 1);  // 0 .. NGATHER-1
+        const int x = gt & 7, r8 = (gt >> 3) & 7;
+        uint32_t dst_off[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) dst_off[k] = ((gt >> 6) + 4 * k) * 1024 + r8 * 128 + ((x ^ r8) << 4);
         uint32_t ring_n = 0;  // chunks filled so far
-        int q_n = 0, qi_n = 0;
-        auto gather_chunk = [&](const uint8_t* base, int row_bytes, int chunk, const int32_t* lst, int tile, int n) {
-            // one 128-row x 128-byte chunk of the keys of `tile` into the next ring slot
-            const int s = static_cast<int>(ring_n % NS);
-            const bool go = mbar_wait(bar_ring_empty(s), ((ring_n / NS) & 1) ^ 1, abort_flag);
-            if (go) {
-                const uint32_t dst0 = s_base + Cfg::OFF_RING + s * Cfg::CH_BYTES;
-                for (int u = ptid; u < Cfg::BM * 8; u += NPROD) {
-                    const int r = u >> 3, x = u & 7;
-                    const int slot = tile * Cfg::BM + r;
+        for (int r = 0; r < n_rounds; ++r) {
+            const int row = row_of(r);
+            if (row < 0) continue;
+            const int buf = r & 1;
+            mbar_wait(bar_list_full(buf), (r >> 1) & 1, abort_flag);
+            const int n = misc_s[buf];
+            if (n == 0) continue;
+            const int32_t* lst = list_s + buf * Cfg::MAX_TOPK;
+            const int T = dist_tiles(n);
+            const int b = row / p.n_q;
+            // the `nch` 128-byte chunks of the keys of `tile`, one ring slot each
+            auto gather_tile = [&](const uint8_t* base, int row_bytes, int nch, int tile) {
+                const uint8_t* src[4];
+                uint32_t bytes[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int slot = tile * Cfg::BM + (gt >> 3) + 32 * k;
                     const int key = slot < n ? lst[slot] : -1;
-                    const uint8_t* src = base + static_cast<int64_t>(key < 0 ? 0 : key) * row_bytes + chunk * 128 + x * 16;
-                    const uint32_t dst = dst0 + (r >> 3) * 1024 + (r & 7) * 128 + ((x ^ (r & 7)) << 4);
-                    cp_async_16_zfill(dst, src, key < 0 ? 0u : 16u);
+                    src[k] = base + static_cast<int64_t>(key < 0 ? 0 : key) * row_bytes + x * 16;
+                    bytes[k] = key < 0 ? 0u : 16u;
                 }
-                cp_async_mbar_arrive_noinc(bar_ring_full(s));
+                for (int c = 0; c < nch; ++c) {
+                    const int s = static_cast<int>(ring_n % NS);
+                    if (mbar_wait(bar_ring_empty(s), ((ring_n / NS) & 1) ^ 1, abort_flag)) {
+                        const uint32_t dst0 = s_base + Cfg::OFF_RING + s * Cfg::CH_BYTES;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) cp_async_16_zfill(dst0 + dst_off[k], src[k] + c * 128, bytes[k]);
+                        cp_async_mbar_arrive_noinc(bar_ring_full(s));
+                    }
+                    ++ring_n;
+                }
+            };
+            for (int l = 0; l < L; ++l) {
+                const uint8_t* kvb = reinterpret_cast<const uint8_t*>(p.kv[l] + static_cast<int64_t>(b) * p.n_k * DQK);
+                for (int t = 0; t < T; ++t) gather_tile(kvb, DQK * 2, NCH, t);
             }
-            ++ring_n;
-        };
+            const int ibytes = Cfg::DI * (Cfg::FP8I ? 1 : 2);
+            const uint8_t* kib = reinterpret_cast<const uint8_t*>(p.k_I) + static_cast<int64_t>(b) * p.n_k * ibytes;
+            for (int t = 0; t < T; ++t) gather_tile(kib, ibytes, NCH_I, t);
+        }
+        cp_async_wait_all();
+        } else {
+        // ------------------- index compaction, query rows and L2 prefetches
+        const int at = threadIdx.x - 32 * Cfg::AUX_WARP0;  // 0 .. NAUX-1
+        const int aw = at >> 5;
+        constexpr int NAUX = Cfg::NAUX;
+        int q_n = 0, qi_n = 0;
         // 64 rows of `row_bytes` (a query's heads) into 128-byte swizzled chunks at dst0
         auto load_rows64 = [&](uint32_t dst0, const uint8_t* src0, int row_bytes, uint32_t bar) {
-            const int units = 64 * (row_bytes / 16);
-            for (int u = ptid; u < units; u += NPROD) {
-                const int h = u / (row_bytes / 16), c16 = u % (row_bytes / 16);
-                const int ch = c16 >> 3, x = c16 & 7;
-                const uint32_t dst = dst0 + ch * Cfg::Q_CH_BYTES + (h >> 3) * 1024 + (h & 7) * 128 + ((x ^ (h & 7)) << 4);
+            const int upr = row_bytes / 16;  // 16-byte units per row
+            for (int u = at; u < 64 * upr; u += NAUX) {
+                const int h = u / upr, c16 = u % upr;
+                const int ch = c16 >> 3, xx = c16 & 7;
+                const uint32_t dst = dst0 + ch * Cfg::Q_CH_BYTES + (h >> 3) * 1024 + (h & 7) * 128 + ((xx ^ (h & 7)) << 4);
                 cp_async_16(dst, src0 + static_cast<int64_t>(h) * row_bytes + c16 * 16);
             }
             cp_async_mbar_arrive_noinc(bar);
@@ -208,18 +252,18 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) distill_tc_kernel(const __gri
             // ordered compaction of the valid entries of the index row
             const int32_t* irow = p.idx + static_cast<int64_t>(row) * p.topk;
             int run = 0;
-            for (int e0 = 0; e0 < p.topk; e0 += NPROD) {
-                const int e = e0 + ptid;
+            for (int e0 = 0; e0 < p.topk; e0 += NAUX) {
+                const int e = e0 + at;
                 const int s = e < p.topk ? irow[e] : -1;
                 const bool ok = s >= 0 && s < p.n_k;
                 const uint32_t bal = __ballot_sync(0xffffffffu, ok);
-                if (lane == 0) misc_s[8 + pw] = __popc(bal);
-                named_bar_sync(2, NPROD);
+                if (lane == 0) misc_s[8 + aw] = __popc(bal);
+                named_bar_sync(2, NAUX);
                 int before = 0, total = 0;
 #pragma unroll
-                for (int w = 0; w < NPROD / 32; ++w) {
+                for (int w = 0; w < NAUX / 32; ++w) {
                     const int c = misc_s[8 + w];
-                    before += w < pw ? c : 0;
+                    before += w < aw ? c : 0;
                     total += c;
                 }
                 if (ok) {
@@ -227,42 +271,47 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) distill_tc_kernel(const __gri
                     if (IC_DCHECK(slot < Cfg::MAX_TOPK)) lst[slot] = s;
                 }
                 run += total;
-                named_bar_sync(2, NPROD);  // misc_s is rewritten by the next chunk
+                named_bar_sync(2, NAUX);  // misc_s is rewritten by the next chunk
             }
             const int n = run;
-            if (ptid == 0) {
+            if (at == 0) {
                 misc_s[buf] = n;
                 mbar_arrive(bar_list_full(buf));  // release: the list and its count
             }
             if (n == 0) continue;
-            const int T = dist_tiles(n);
             const int b = row / p.n_q;
+            // every layer's query rows and selected key rows are requested from L2
+            // ahead of their loads
+            {
+                const int ib = Cfg::DI * (Cfg::FP8I ? 1 : 2);
+                for (int u = at; u <= L; u += NAUX) {
+                    if (u < L)
+                        prefetch_l2_bulk(p.q[u] + static_cast<int64_t>(row) * Cfg::H * DQK, Cfg::H * DQK * 2);
+                    else
+                        prefetch_l2_bulk(reinterpret_cast<const uint8_t*>(p.q_I) + static_cast<int64_t>(row) * Cfg::HI * ib,
+                                         Cfg::HI * ib);
+                }
+            }
             for (int l = 0; l < L; ++l) {
                 const uint8_t* kvb = reinterpret_cast<const uint8_t*>(p.kv[l] + static_cast<int64_t>(b) * p.n_k * DQK);
-                // the layer's selected rows are requested from L2 ahead of the gathers
-                for (int j = ptid; j < n; j += NPROD) prefetch_l2_bulk(kvb + static_cast<int64_t>(lst[j]) * DQK * 2, DQK * 2);
+                for (int j = at; j < n; j += NAUX) prefetch_l2_bulk(kvb + static_cast<int64_t>(lst[j]) * DQK * 2, DQK * 2);
+            }
+            for (int l = 0; l < L; ++l) {
                 if (mbar_wait(bar_q_empty, (q_n & 1) ^ 1, abort_flag))
                     load_rows64(s_base + Cfg::OFF_Q,
                                 reinterpret_cast<const uint8_t*>(p.q[l] + static_cast<int64_t>(row) * Cfg::H * DQK), DQK * 2,
                                 bar_q_full);
                 ++q_n;
-                for (int t = 0; t < T; ++t)
-                    for (int c = 0; c < NCH; ++c) gather_chunk(kvb, DQK * 2, c, lst, t, n);
-                for (int t = 0; t < dist_recompute<Cfg>(T); ++t)
-                    for (int c = 0; c < NCH; ++c) gather_chunk(kvb, DQK * 2, c, lst, t, n);
             }
-            // the indexer's keys
             const int ibytes = Cfg::DI * (Cfg::FP8I ? 1 : 2);
-            const uint8_t* kib = reinterpret_cast<const uint8_t*>(p.k_I) + static_cast<int64_t>(b) * p.n_k * ibytes;
             if (mbar_wait(bar_qi_empty, (qi_n & 1) ^ 1, abort_flag))
                 load_rows64(s_base + Cfg::OFF_QI,
                             reinterpret_cast<const uint8_t*>(p.q_I) + static_cast<int64_t>(row) * Cfg::HI * ibytes, ibytes,
                             bar_qi_full);
             ++qi_n;
-            for (int t = 0; t < T; ++t)
-                for (int c = 0; c < NCH_I; ++c) gather_chunk(kib, ibytes, c, lst, t, n);
         }
         cp_async_wait_all();
+        }
       } else if (lane == 0) {
         // ------------------------------------------------------ MMA issuer
         uint32_t ring_n = 0, job = 0;
@@ -307,8 +356,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) distill_tc_kernel(const __gri
                 mbar_wait(bar_q_full, q_n & 1, abort_flag);
                 tc_fence_after();
                 ++q_n;
-                const int jobs = T + dist_recompute<Cfg>(T);
-                for (int t = 0; t < jobs; ++t) run_job(NCH, s_base + Cfg::OFF_Q, Cfg::IDESC_S, false);
+                for (int t = 0; t < T; ++t) run_job(NCH, s_base + Cfg::OFF_Q, Cfg::IDESC_S, false);
                 mma_commit(bar_q_empty);  // the query rows may be replaced
             }
             mbar_wait(bar_qi_full, qi_n & 1, abort_flag);
@@ -325,6 +373,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) distill_tc_kernel(const __gri
         const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
         const float c_log2 = p.sm_scale * 1.4426950408889634f;
         const float inv_norm = 1.f / (static_cast<float>(Cfg::H) * static_cast<float>(L));
+        float4* spill = reinterpret_cast<float4*>(static_cast<uint8_t*>(p.spill) + Cfg::SPILL_BYTES_PER_CTA * blockIdx.x);
         uint32_t job = 0;
         auto acquire = [&](uint32_t j) {
             mbar_wait(bar_acc_full(static_cast<int>(j % NSLOT)), (j / NSLOT) & 1, abort_flag);
@@ -362,14 +411,23 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) distill_tc_kernel(const __gri
                         ls[h] = 0.f;
                     }
                     const uint32_t job0 = job;
+                    const int R = dist_spilled<Cfg>(T);
                     for (int t = 0; t < T; ++t) {
                         const uint32_t ta = acquire(job0 + t);
                         const bool valid = t * Cfg::BM + tid < n;
+                        float4* sp = spill + static_cast<size_t>(t) * 16 * Cfg::BM + tid;
 #pragma unroll
                         for (int half = 0; half < 2; ++half) {
                             uint32_t v[32];
                             tmem_ld<32>(ta + half * 32, v);
                             tmem_wait_ld();
+                            if (t < R) {  // this tile's logits wait in the workspace
+#pragma unroll
+                                for (int g = 0; g < 8; ++g)
+                                    sp[(half * 8 + g) * Cfg::BM] =
+                                        make_float4(__uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1]),
+                                                    __uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]));
+                            }
                             if (valid) {
 #pragma unroll
                                 for (int k = 0; k < 32; ++k) {
@@ -383,7 +441,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) distill_tc_kernel(const __gri
                                 }
                             }
                         }
-                        if (t < T - Cfg::RESIDENT) release(job0 + t);
+                        if (t < R) release(job0 + t);
                     }
                     // merge across the warp (a butterfly that halves the heads
                     // held per lane at each step: lane L ends with heads 2L, 2L+1)
@@ -427,8 +485,26 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) distill_tc_kernel(const __gri
                         hl_s[tid] = ll > 0.f ? 1.f / ll : 0.f;
                     }
                     named_bar_sync(1, 128);
-                    // ---- probability pass: resident tiles, then the recomputed ones
-                    auto prob_tile = [&](uint32_t j, int t) {
+                    // ---- probability pass: resident tiles from tensor memory, then
+                    // the spilled ones from the workspace (the next tile's loads in
+                    // flight while one is summed)
+                    // sum over heads g0 .. g0+31 of 2^(z - max) / sum; z4(i) gives
+                    // the logits of heads g0 + 4i .. g0 + 4i + 3
+                    auto prob_sum = [&](auto&& z4, int g0, float acc) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float4 z = z4(i);
+                            const float4 hm = *reinterpret_cast<const float4*>(hm_s + g0 + 4 * i);
+                            const float4 hl = *reinterpret_cast<const float4*>(hl_s + g0 + 4 * i);
+                            acc = fmaf(ex2_approx(fmaf(z.x, c_log2, -hm.x)), hl.x, acc);
+                            acc = fmaf(ex2_approx(fmaf(z.y, c_log2, -hm.y)), hl.y, acc);
+                            acc = fmaf(ex2_approx(fmaf(z.z, c_log2, -hm.z)), hl.z, acc);
+                            acc = fmaf(ex2_approx(fmaf(z.w, c_log2, -hm.w)), hl.w, acc);
+                        }
+                        return acc;
+                    };
+                    for (int t = R; t < T; ++t) {
+                        const uint32_t j = job0 + t;
                         const uint32_t ta = tmem_base + lane_base + static_cast<uint32_t>(j % NSLOT) * 64;
                         float acc = 0.f;
 #pragma unroll
@@ -436,27 +512,39 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1) distill_tc_kernel(const __gri
                             uint32_t v[32];
                             tmem_ld<32>(ta + half * 32, v);
                             tmem_wait_ld();
-#pragma unroll
-                            for (int k = 0; k < 32; k += 4) {
-                                const float4 hm = *reinterpret_cast<const float4*>(hm_s + half * 32 + k);
-                                const float4 hl = *reinterpret_cast<const float4*>(hl_s + half * 32 + k);
-                                acc = fmaf(ex2_approx(fmaf(__uint_as_float(v[k + 0]), c_log2, -hm.x)), hl.x, acc);
-                                acc = fmaf(ex2_approx(fmaf(__uint_as_float(v[k + 1]), c_log2, -hm.y)), hl.y, acc);
-                                acc = fmaf(ex2_approx(fmaf(__uint_as_float(v[k + 2]), c_log2, -hm.z)), hl.z, acc);
-                                acc = fmaf(ex2_approx(fmaf(__uint_as_float(v[k + 3]), c_log2, -hm.w)), hl.w, acc);
-                            }
+                            acc = prob_sum(
+                                [&](int i) {
+                                    return make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                                       __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+                                },
+                                half * 32, acc);
                         }
                         release(j);
                         const int slot = t * Cfg::BM + tid;
                         if (slot < n) P_s[slot] += acc * inv_norm;
-                    };
-                    const int R = dist_recompute<Cfg>(T);
-                    for (int t = R; t < T; ++t) prob_tile(job0 + t, t);
-                    for (int t = 0; t < R; ++t) {
-                        acquire(job0 + T + t);
-                        prob_tile(job0 + T + t, t);
                     }
-                    job = job0 + T + R;
+                    if (R > 0) {
+                        // half tiles (32 heads, 8 float4) in order, each loaded one
+                        // half ahead of its sum
+                        float4 cur[8];
+#pragma unroll
+                        for (int g = 0; g < 8; ++g) cur[g] = spill[g * Cfg::BM + tid];
+                        for (int t = 0; t < R; ++t) {
+                            const float4* sp = spill + static_cast<size_t>(t) * 16 * Cfg::BM + tid;
+                            float4 nxt[8];
+#pragma unroll
+                            for (int g = 0; g < 8; ++g) nxt[g] = sp[(8 + g) * Cfg::BM];
+                            float acc = prob_sum([&](int i) { return cur[i]; }, 0, 0.f);
+                            if (t + 1 < R) {
+#pragma unroll
+                                for (int g = 0; g < 8; ++g) cur[g] = sp[(16 + g) * Cfg::BM];
+                            }
+                            acc = prob_sum([&](int i) { return nxt[i]; }, 32, acc);
+                            const int slot = t * Cfg::BM + tid;
+                            if (slot < n) P_s[slot] += acc * inv_norm;
+                        }
+                    }
+                    job = job0 + T;
                 }
                 // ---- the indexer's scores of the same keys
                 for (int t = 0; t < T; ++t) {

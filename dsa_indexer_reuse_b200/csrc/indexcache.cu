@@ -545,17 +545,28 @@ ic_status launch_distill(const ic::DistillParams& p, int rows, cudaStream_t stre
     return IC_OK;
 }
 
+// The model's shapes run on the tensor cores; other shapes on the CUDA cores.
+bool distill_on_tensor_cores(int H, int d_qk, int H_I, int d_I) {
+    return H == 64 && d_qk == 576 && H_I == 64 && d_I == 128;
+}
+
+// Grid of the tensor-core kernel (persistent CTAs, one query row at a time)
+// and its workspace: the spilled logits of up to SPILL_TILES tiles per CTA
+// (only rows of more than RESIDENT tiles, i.e. topk > 1024, spill).
+using DistTcAny = ic::DistTcCfg<576, true>;
+static_assert(DistTcAny::SPILL_BYTES_PER_CTA == ic::DistTcCfg<576, false>::SPILL_BYTES_PER_CTA, "spill size");
+int distill_tc_grid(int rows, int sms) { return std::max(1, std::min(rows, sms)); }
+size_t distill_tc_ws_bytes(int rows, int topk, int sms) {
+    if (topk <= DistTcAny::RESIDENT * DistTcAny::BM) return 0;
+    return DistTcAny::SPILL_BYTES_PER_CTA * static_cast<size_t>(distill_tc_grid(rows, sms));
+}
+
 template <class Cfg>
-ic_status launch_distill_tc(const ic::DistillParams& p, cudaStream_t stream) {
+ic_status launch_distill_tc(const ic::DistillParams& p, int sms, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(ic::distill_tc_kernel<Cfg>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Cfg::SMEM_ALLOC);
     if (e != cudaSuccess) return cuda_fail("distill (tensor cores) smem attribute", e);
-    int dev = 0, sms = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return cuda_fail("cudaGetDevice", e);
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-        return cuda_fail("SM count", e);
-    const int grid = std::max(1, std::min(p.rows, sms));
-    ic::distill_tc_kernel<Cfg><<<grid, Cfg::THREADS, Cfg::SMEM_ALLOC, stream>>>(p);
+    ic::distill_tc_kernel<Cfg><<<distill_tc_grid(p.rows, sms), Cfg::THREADS, Cfg::SMEM_ALLOC, stream>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("distill (tensor cores) launch", e);
     return IC_OK;
@@ -1145,11 +1156,25 @@ ic_status ic_layer_stack_host(const ic_layer_io* layers, int n_layers, int index
 }
 
 
+ic_status ic_distill_target_workspace_size(int batch, int n_q, int topk, int H, int d_qk, int H_I, int d_I,
+                                           size_t* bytes_out) {
+    if (!bytes_out || batch < 0 || n_q < 0 || topk <= 0 || H <= 0 || d_qk <= 0 || H_I <= 0 || d_I <= 0)
+        return IC_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(batch) * n_q > std::numeric_limits<int>::max()) return IC_ERR_UNSUPPORTED;
+    *bytes_out = 0;
+    if (!distill_on_tensor_cores(H, d_qk, H_I, d_I) || topk > 2048) return IC_OK;
+    const DeviceInfo dev = device_info();
+    if (dev.sms <= 0) return cuda_fail("device query", cudaErrorNoDevice);
+    *bytes_out = distill_tc_ws_bytes(batch * n_q, topk, dev.sms);
+    return IC_OK;
+}
+
 ic_status ic_distill_target(const void* const* q_layers, const void* const* kv_layers, int n_served,
                             const void* q_I, const float* q_scale, const void* w, ic_dtype w_dtype,
                             const void* k_I, const float* k_scale, ic_dtype qk_dtype, const int32_t* idx,
                             int batch, int n_q, int n_k, int H_I, int d_I, int topk, int H, int d_qk,
-                            float sm_scale, float* target_out, float* kl_out, void* stream) {
+                            float sm_scale, float* target_out, float* kl_out, void* workspace,
+                            size_t workspace_bytes, void* stream) {
     if (batch < 0 || n_q < 0 || n_k < 0 || topk <= 0 || H <= 0 || d_qk <= 0 || H_I <= 0 || d_I <= 0)
         return IC_ERR_INVALID_ARG;
     if (n_served < 1 || !q_layers || !kv_layers) return IC_ERR_INVALID_ARG;
@@ -1162,7 +1187,7 @@ ic_status ic_distill_target(const void* const* q_layers, const void* const* kv_l
     if (batch == 0 || n_q == 0) return IC_OK;
     if (!q_I || !w || !idx || !kl_out || (n_k > 0 && !k_I)) return IC_ERR_INVALID_ARG;
     if (qk_dtype == IC_FP8_E4M3 && (!q_scale || (n_k > 0 && !k_scale))) return IC_ERR_INVALID_ARG;
-    if (!aligned16(k_I)) return IC_ERR_INVALID_ARG;
+    if (!aligned16(k_I) || !aligned16(q_I)) return IC_ERR_INVALID_ARG;
     ic::DistillParams p{};
     for (int l = 0; l < n_served; ++l) {
         if (!q_layers[l] || (n_k > 0 && !kv_layers[l])) return IC_ERR_INVALID_ARG;
@@ -1192,9 +1217,15 @@ ic_status ic_distill_target(const void* const* q_layers, const void* const* kv_l
     const cudaStream_t cs = static_cast<cudaStream_t>(stream);
     // the model's shapes (64 heads over 576-wide latent rows, a 64-head
     // 128-wide indexer) run on the tensor cores; other shapes on the CUDA cores
-    if (H == 64 && d_qk == 576 && H_I == 64 && d_I == 128 && aligned16(q_I))
-        return p.fp8 ? launch_distill_tc<ic::DistTcCfg<576, true>>(p, cs)
-                     : launch_distill_tc<ic::DistTcCfg<576, false>>(p, cs);
+    if (distill_on_tensor_cores(H, d_qk, H_I, d_I)) {
+        const DeviceInfo dev = device_info();
+        if (dev.sms <= 0) return cuda_fail("device query", cudaErrorNoDevice);
+        const size_t need = distill_tc_ws_bytes(rows, topk, dev.sms);
+        if (need > 0 && (!workspace || workspace_bytes < need || !aligned256(workspace))) return IC_ERR_WORKSPACE;
+        p.spill = workspace;
+        return p.fp8 ? launch_distill_tc<ic::DistTcCfg<576, true>>(p, dev.sms, cs)
+                     : launch_distill_tc<ic::DistTcCfg<576, false>>(p, dev.sms, cs);
+    }
     if (d_qk == 576) return H_I == 64 ? launch_distill<576, 64>(p, rows, cs) : launch_distill<576, 4>(p, rows, cs);
     return H_I == 64 ? launch_distill<64, 64>(p, rows, cs) : launch_distill<64, 4>(p, rows, cs);
 }

@@ -282,14 +282,23 @@ ic_status ic_layer_stack_host(const ic_layer_io* layers, int n_layers, int index
  *           no valid position)
  * fp32 arithmetic. Supported: 1 <= n_served <= 64, d_qk in {64, 576},
  * 1 <= H <= 64, H_I in {4, 64}, d_I a multiple of 8 (<= 128), topk <= 2048;
- * others IC_ERR_UNSUPPORTED. Asynchronous on `stream`; no workspace.
+ * others IC_ERR_UNSUPPORTED. The model's shapes (H = 64, d_qk = 576,
+ * H_I = 64, d_I = 128) run on the tensor cores and, for topk > 1024, need
+ * workspace (ic_distill_target_workspace_size bytes, 256-byte aligned; else
+ * IC_ERR_WORKSPACE): logits of up to 8 tiles of 128 keys per CTA wait there
+ * between a statistics pass and a probability pass. Other shapes need none
+ * (workspace may be NULL). q_I, k_I and the q/kv pointers 16-byte aligned.
+ * Asynchronous on `stream`.
  */
+ic_status ic_distill_target_workspace_size(int batch, int n_q, int topk, int H, int d_qk, int H_I, int d_I,
+                                           size_t* bytes_out);
 ic_status ic_distill_target(const void* const* q_layers, const void* const* kv_layers, int n_served,
                             const void* q_I, const float* q_scale, const void* w, ic_dtype w_dtype,
                             const void* k_I, const float* k_scale, ic_dtype qk_dtype,
                             const int32_t* idx, int batch, int n_q, int n_k, int H_I, int d_I,
                             int topk, int H, int d_qk, float sm_scale, float* target_out,
-                            float* kl_out, void* stream);
+                            float* kl_out, void* workspace,
+                            size_t workspace_bytes, void* stream);
 
 /*
  * Pattern tools (IndexCache paper, Appendix Figure 4: the pairwise top-k

@@ -169,7 +169,7 @@ def test_distill_target_validates_on_the_host(ic):
         return lib.ic_distill_target(ctypes.cast(arr, ctypes.c_void_p), ctypes.cast(arr, ctypes.c_void_p),
                                      n_served, q.ctypes.data, None, q.ctypes.data, w, q.ctypes.data, None,
                                      qk, idx.ctypes.data, batch, 4, 64, H_I, d_I, topk, H, d_qk, 0.125,
-                                     None, kl_ptr, None)
+                                     None, kl_ptr, None, 0, None)
     assert call(n_served=0) == 1                      # IC_ERR_INVALID_ARG
     assert call(kl_ptr=None) == 1
     assert call(qk=7) == 1 and call(w=1) == 1         # FP8 weights are not a w dtype
@@ -178,3 +178,15 @@ def test_distill_target_validates_on_the_host(ic):
     assert call(d_qk=128) == 3 and call(H=65) == 3 and call(topk=4096) == 3
     assert call(H_I=8) == 3 and call(d_I=60) == 3
     assert call(batch=0) == 0                         # nothing to do
+
+
+def test_distill_workspace_size_on_the_host(ic):
+    """Shapes outside the tensor-core configuration need no workspace; the
+    size query checks its arguments without touching a device."""
+    lib = ic.lib
+    out = ctypes.c_size_t(123)
+    assert lib.ic_distill_target_workspace_size(1, 64, 2048, 4, 64, 4, 64, ctypes.byref(out)) == 0
+    assert out.value == 0
+    assert lib.ic_distill_target_workspace_size(1, 64, 2048, 4, 64, 4, 64, None) == 1
+    assert lib.ic_distill_target_workspace_size(-1, 64, 2048, 64, 576, 64, 128, ctypes.byref(out)) == 1
+    assert lib.ic_distill_target_workspace_size(1, 64, 0, 64, 576, 64, 128, ctypes.byref(out)) == 1

@@ -119,3 +119,25 @@ def test_latent_long_rows_peaked_logits(cuda_ok):
     ind, served, idx = _inputs(wl, 2, seed=12)
     served = [(q * 32, kv) for q, kv in served]
     _check(wl, ind, served, idx)
+
+
+def test_workspace_is_required_for_long_rows(cuda_ok):
+    # topk 2048 on the tensor-core shapes spills logits: without a workspace
+    # the call is refused before anything is enqueued
+    import ctypes
+    wl = W.DECODE_32X32K.with_(batch=1, n_k=1536, q_pos0=1535, n_layers=1)
+    ind, served, idx = _inputs(wl, 1, seed=14)
+    need = ic.distill_target_workspace_size(1, 1, wl.topk, wl.H, wl.d_qk, wl.H_I, wl.d_I)
+    assert need > 0
+    (q, kv), = served
+    q_arr = (ctypes.c_void_p * 1)(q.data_ptr())
+    kv_arr = (ctypes.c_void_p * 1)(kv.data_ptr())
+    kl = torch.empty(1, dtype=torch.float32, device="cuda")
+    small = torch.empty(need // 2, dtype=torch.uint8, device="cuda")
+    for ws, n in ((None, 0), (small.data_ptr(), small.numel())):
+        code = ic.lib.ic_distill_target(ctypes.cast(q_arr, ctypes.c_void_p), ctypes.cast(kv_arr, ctypes.c_void_p),
+                                        1, ind["q_I"].data_ptr(), ind["q_scale"].data_ptr(), ind["w"].data_ptr(),
+                                        2 if ind["w"].dtype == torch.float32 else 0, ind["k_I"].data_ptr(),
+                                        ind["k_scale"].data_ptr(), 1, idx.data_ptr(), 1, 1, wl.n_k, wl.H_I, wl.d_I,
+                                        wl.topk, wl.H, wl.d_qk, wl.sm_scale, None, kl.data_ptr(), ws, n, None)
+        assert code == 6  # IC_ERR_WORKSPACE
