@@ -370,8 +370,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 // stage, whose refill (tile j+1) then overlaps the rest of QK(j).
                 auto pv_ready = [&](int j) {
                     const int s = pv_n & 1;
-                    return mbar_try_wait(bar_p_full(s), (pv_n >> 1) & 1) &&
-                           (j != 1 || mbar_try_wait(bar_o_free, (q_n & 1) ^ 1));
+                    return mbar_test_wait(bar_p_full(s), (pv_n >> 1) & 1) &&
+                           (j != 1 || mbar_test_wait(bar_o_free, (q_n & 1) ^ 1));
                 };
                 auto issue_pv = [&](int j) {
                     // O^T += V^T . P^T for tile j-1
