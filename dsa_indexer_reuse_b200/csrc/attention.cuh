@@ -59,7 +59,6 @@ struct AttnParams {
     float sm_scale_log2;       // sm_scale * log2(e)
     int n_splits;
     int n_work;                // rows * n_splits
-    int prefetch_split;        // 1: L2-prefetch each slice's rows when its work item starts
 };
 
 template <int DQK_, int DV_>
@@ -287,13 +286,6 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 const int row_base = b * p.n_k;
                 const int fallback = list_s[lo];  // rows past the slice end re-read a valid row
                 const __nv_bfloat16* kvb = p.kv + static_cast<int64_t>(row_base) * Cfg::DQK;
-                if (p.prefetch_split) {
-                    // decode-style split: every selected row of this slice is asked of
-                    // L2 at once, so the slice's HBM reads run at full depth while the
-                    // tiles are gathered (from L2) and computed one after another
-                    for (int e = lo + ptid; e < hi; e += Cfg::NPROD)
-                        prefetch_l2_bulk(kvb + static_cast<int64_t>(list_s[e]) * Cfg::DQK, Cfg::DQK * 2);
-                }
                 for (int j = 0; j < n_tiles; ++j) {
                     const int s = kv_n & 1;
                     const bool issue = mbar_wait(bar_kv_empty(s), ((kv_n >> 1) & 1) ^ 1, abort_flag);

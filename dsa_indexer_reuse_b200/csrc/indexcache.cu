@@ -107,7 +107,12 @@ cudaError_t launch(const void* kernel, dim3 grid, dim3 block, size_t smem, cudaS
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
+#ifdef IC_NO_PDL
+    cfg.numAttrs = 0;
+    (void)pdl;
+#else
     cfg.numAttrs = pdl ? 1 : 0;
+#endif
     return cudaLaunchKernelExC(&cfg, kernel, args);
 }
 bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
@@ -464,10 +469,6 @@ ic_status launch_attn(const void* q, const void* kv, const int32_t* idx, int bat
     p.sm_scale_log2 = sm_scale * 1.4426950408889634f;
     p.n_splits = splits;
     p.n_work = rows * splits;
-    // decode-style calls read their rows from HBM: every slice is prefetched into
-    // L2 up front when all the launch's selected rows fit in a part of L2
-    const double sel_bytes = static_cast<double>(rows) * topk * d_qk * 2;
-    p.prefetch_split = (splits > 1 && sel_bytes <= 80e6) ? 1 : 0;
     if (check_register_pool(pl.kernel, pl.regs) != IC_OK)
         return cuda_fail("attention register pool", cudaErrorInvalidConfiguration);
     cudaError_t e = cudaFuncSetAttribute(pl.kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem);
