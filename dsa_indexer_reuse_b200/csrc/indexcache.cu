@@ -21,6 +21,7 @@
 
 #include "../../include/indexcache.h"
 #include "attention.cuh"
+#include "attention_pair.cuh"
 #include "common.cuh"
 #include "indexer.cuh"
 #include "indexer_decode.cuh"
@@ -387,21 +388,30 @@ struct AttnPlan {
     void (*combine)(const float*, const float*, int, int, __nv_bfloat16*) = nullptr;
 };
 
-template <class Cfg>
+// The 576 / 512 latent shape forms the scores of two 64-key tiles per MMA
+// chain (attention_pair.cuh); IC_ATTN_PAIR=0 selects the one-tile kernel.
+#ifndef IC_ATTN_PAIR
+#define IC_ATTN_PAIR 1
+#endif
+
+template <class Cfg, bool PAIR = false>
 AttnPlan attn_plan() {
     AttnPlan pl;
     pl.smem = Cfg::SMEM_ALLOC;
     pl.threads = Cfg::THREADS;
     pl.dv = Cfg::DV;
     pl.regs = 65536 / Cfg::THREADS;
-    pl.kernel = reinterpret_cast<const void*>(&ic::sparse_attn_kernel<Cfg>);
+    if constexpr (PAIR)
+        pl.kernel = reinterpret_cast<const void*>(&ic::sparse_attn_pair_kernel<Cfg>);
+    else
+        pl.kernel = reinterpret_cast<const void*>(&ic::sparse_attn_kernel<Cfg>);
     pl.combine = &ic::attn_combine_kernel<Cfg::DV>;
     return pl;
 }
 
 bool choose_attn_plan(int d_qk, int d_v, AttnPlan* pl) {
     if (d_qk == 576 && d_v == 512) {
-        *pl = attn_plan<Attn576>();
+        *pl = attn_plan<Attn576, IC_ATTN_PAIR != 0>();
         return true;
     }
     if (d_qk == 64 && d_v == 64) {
