@@ -455,6 +455,9 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
               float ksc_f = scale_of(s_key);
               int till_meet = per;
               if (wk.n_tiles > 0) issue_loads(ait);
+              // two tiles per loop trip: the loop's bookkeeping is a measurable
+              // share of the epilogue's issue slots
+#pragma unroll 2
               for (int t = 0; t < wk.n_tiles; ++t, ++ait, s_key += IDX_BM) {
                 const int a = ait & 1;
                 // the next tile's key scale is requested a whole tile ahead
