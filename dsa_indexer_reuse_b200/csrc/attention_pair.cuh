@@ -327,11 +327,19 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 // z = logit (log2 units) minus the per-head reference, in place
                 float zmax = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    const float z = __fmul_rn(__uint_as_float(sv[c]), p.sm_scale_log2) - m_s[hb + c];
-                    zmax = fmaxf(zmax, valid ? z : -INFINITY);
-                    sv[c] = __float_as_uint(z);
+                for (int c = 0; c < 32; c += 4) {
+                    const float4 m4 = *reinterpret_cast<const float4*>(m_s + hb + c);
+                    const float z0 = fmaf(__uint_as_float(sv[c + 0]), p.sm_scale_log2, -m4.x);
+                    const float z1 = fmaf(__uint_as_float(sv[c + 1]), p.sm_scale_log2, -m4.y);
+                    const float z2 = fmaf(__uint_as_float(sv[c + 2]), p.sm_scale_log2, -m4.z);
+                    const float z3 = fmaf(__uint_as_float(sv[c + 3]), p.sm_scale_log2, -m4.w);
+                    zmax = fmaxf(zmax, fmaxf(fmaxf(z0, z1), fmaxf(z2, z3)));
+                    sv[c + 0] = __float_as_uint(z0);
+                    sv[c + 1] = __float_as_uint(z1);
+                    sv[c + 2] = __float_as_uint(z2);
+                    sv[c + 3] = __float_as_uint(z3);
                 }
+                if (!valid) zmax = -INFINITY;
                 if (named_bar_or(sbar, 128, zmax > IC_ATTN_RESCALE_LOG2)) {
                     // rare path: raise the reference to the pair's maximum and
                     // rescale the accumulated output and row sums. Every P.V issued
