@@ -27,6 +27,11 @@
 
 #include "attention.cuh"
 
+// setmaxnreg split of the paired kernel (softmax warpgroups / the rest)
+#ifndef IC_ATTN_PAIR_REGS_SMX
+#define IC_ATTN_PAIR_REGS_SMX 152
+#endif
+
 namespace ic {
 
 template <class Cfg>
@@ -34,6 +39,8 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                             const AttnParams p) {
     static_assert(Cfg::DQK == 576 && Cfg::DV == 512 && Cfg::TMA_CH == 0 && Cfg::P_IN_ROPE, "paired tiles: 576 / 512");
+    static_assert(IC_ATTN_PAIR_REGS_SMX % 8 == 0 && IC_ATTN_PAIR_REGS_SMX >= 136 && IC_ATTN_PAIR_REGS_SMX <= 176,
+                  "register split");
     constexpr int PCH = 2 * Cfg::CH_BYTES;  // one chunk slot: chunk c of both stages
     constexpr uint32_t IDESC_S2 = make_idesc(128, Cfg::NH, FMT_BF16, FMT_BF16);
     extern __shared__ uint8_t smem_raw[];
@@ -97,7 +104,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     uint32_t q_armed = 0, kv_armed[2] = {0u, 0u};
 
     if (warp >= 8) {
-      regs_dec<Cfg::REGS_OTHER>();
+      regs_dec<256 - IC_ATTN_PAIR_REGS_SMX>();
       if (warp != MMA_WARP) {
         // ------------------------------ index compaction + cp.async row gathers
         const int pw = warp < MMA_WARP ? warp - 8 : warp - 9;  // producer warp 0..6
@@ -278,7 +285,7 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
         }
       }
     } else {
-        regs_inc<Cfg::REGS_SOFTMAX>();
+        regs_inc<IC_ATTN_PAIR_REGS_SMX>();
         // ------------------------------------------------- softmax and output
         const int wq = warp & 3;               // TMEM lane quarter: keys 32 wq .. 32 wq + 31 of a pair
         const int sw = warp >> 2;              // softmax warpgroup
@@ -395,13 +402,18 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 }
                 // probabilities, row sums, and this key's bf16 P^T row (heads hb .. hb+31)
                 uint32_t packed[16];
+                if (valid) {  // uniform per thread: only a slice's last tile has invalid keys
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float p0 = valid ? ex2_approx(__uint_as_float(sv[2 * i])) : 0.f;
-                    const float p1 = valid ? ex2_approx(__uint_as_float(sv[2 * i + 1])) : 0.f;
-                    l_part[2 * i] += p0;
-                    l_part[2 * i + 1] += p1;
-                    packed[i] = pack_bf16x2(p0, p1);
+                    for (int i = 0; i < 16; ++i) {
+                        const float p0 = ex2_approx(__uint_as_float(sv[2 * i]));
+                        const float p1 = ex2_approx(__uint_as_float(sv[2 * i + 1]));
+                        l_part[2 * i] += p0;
+                        l_part[2 * i + 1] += p1;
+                        packed[i] = pack_bf16x2(p0, p1);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) packed[i] = 0u;
                 }
                 if (has_tile) {
                     const uint32_t prow = s_base + Cfg::OFF_T + Cfg::P_CHUNK * PCH + ps * Cfg::CH_BYTES +
