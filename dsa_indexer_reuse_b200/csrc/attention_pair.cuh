@@ -176,26 +176,36 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
                 const __nv_bfloat16* kvb = p.kv + static_cast<int64_t>(row_base) * Cfg::DQK;
                 for (int j = 0; j < n_tiles; ++j) {
                     const int s = j & 1;  // tile j of a row lives in stage j % 2
+                    // warp pw takes rows pw, pw+NW, ...; their source rows are looked
+                    // up before the wait for the stage, off the refill's critical path
+                    constexpr int NW = Cfg::NPROD / 32;
+                    constexpr int RPW = (Cfg::BK + NW - 1) / NW;  // rows per warp
+                    constexpr int UPR = Cfg::NCH * 8;
+                    constexpr int UPL = (UPR + 31) / 32;
+                    const __nv_bfloat16* src[RPW];
+#pragma unroll
+                    for (int i = 0; i < RPW; ++i) {
+                        const int rr = pw + NW * i;
+                        const int e = lo + j * Cfg::BK + rr;
+                        int key = (rr < Cfg::BK && e < hi) ? list_s[e] : fallback;
+                        if (!IC_DCHECK(key >= 0 && key < p.n_k)) key = 0;
+                        src[i] = kvb + static_cast<int64_t>(key) * Cfg::DQK;
+                    }
                     if (mbar_wait(bar_kv_empty(s), (ku[s] & 1) ^ 1, abort_flag)) {
                         kv_armed[s] = ku[s] + 1;
-                        // warp pw takes rows pw, pw+NW, ...; a row's 72 16-byte units
-                        // go to its chunk slots, 128-byte swizzled
-                        constexpr int NW = Cfg::NPROD / 32;
-                        constexpr int UPR = Cfg::NCH * 8;
-                        constexpr int UPL = (UPR + 31) / 32;
+                        // a row's 72 16-byte units go to its chunk slots, 128-byte swizzled
                         const uint32_t stage = s_base + Cfg::OFF_T + s * Cfg::CH_BYTES;
-                        for (int rr = pw; rr < Cfg::BK; rr += NW) {
-                            const int e = lo + j * Cfg::BK + rr;
-                            int key = e < hi ? list_s[e] : fallback;
-                            if (!IC_DCHECK(key >= 0 && key < p.n_k)) key = 0;
-                            const __nv_bfloat16* src = kvb + static_cast<int64_t>(key) * Cfg::DQK;
+#pragma unroll
+                        for (int i = 0; i < RPW; ++i) {
+                            const int rr = pw + NW * i;
+                            if (rr >= Cfg::BK) break;
                             const uint32_t row_dst = stage + (rr >> 3) * 1024 + (rr & 7) * 128;
                             const int x = rr & 7;
 #pragma unroll
-                            for (int i = 0; i < UPL; ++i) {
-                                const int u = lane + 32 * i;
+                            for (int k = 0; k < UPL; ++k) {
+                                const int u = lane + 32 * k;
                                 if (u < UPR)
-                                    cp_async_16(row_dst + (u >> 3) * PCH + (((u & 7) ^ x) << 4), src + u * 8);
+                                    cp_async_16(row_dst + (u >> 3) * PCH + (((u & 7) ^ x) << 4), src[i] + u * 8);
                             }
                         }
                         cp_async_mbar_arrive_noinc(bar_kv_full(s));
