@@ -122,3 +122,39 @@ def test_deterministic(cuda_ok):
     a, _, _ = run(wl, idx)
     b, _, _ = run(wl, idx)
     assert (a == b).all()
+
+
+def _decode_call(wl, idx, seed, workspace):
+    import dsa_indexer_reuse_b200 as ic
+    att = W.attention_inputs(wl, 0, seed=seed)
+    q, kv = att["q"].cuda(), att["kv"].cuda()
+    out = ic.sparse_attn(q, kv, torch.from_numpy(idx).cuda(), d_v=wl.d_v, sm_scale=wl.sm_scale,
+                         workspace=workspace)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), W.raw_numpy(att["q"]), W.raw_numpy(att["kv"])
+
+
+@pytest.mark.parametrize("shape", ["latent", "tiny_h40"])
+def test_decode_split_dirty_shared_workspace(cuda_ok, shape):
+    # Decode-style calls split each row's keys across CTAs and merge the
+    # partials from the workspace. The workspace starts dirty (every byte
+    # 0xFF), two calls in a row share it, and some rows have no key at all
+    # (every split empty) or keys in the first split only; fewer than 64
+    # heads leave the second softmax warpgroup's head half short.
+    import dsa_indexer_reuse_b200 as ic
+    if shape == "latent":
+        wl = W.DECODE_32X32K.with_(batch=8, n_k=5000, q_pos0=4999)
+    else:
+        wl = W.TINY_INT.with_(batch=8, n_q=1, n_k=5000, q_pos0=4999, topk=1024, H=40)
+    topk = wl.topk
+    assert ic.sparse_attn_workspace_size(wl.batch, 1, wl.H, wl.d_v, topk) > 0  # the split path
+    ws = torch.full((ic.sparse_attn_workspace_size(wl.batch, 1, wl.H, wl.d_v, topk),), 255,
+                    dtype=torch.uint8, device="cuda")
+    for call, seed in enumerate((11, 12)):
+        idx = random_idx(wl.batch, 1, wl.n_k, topk, wl.q_pos0, seed=seed, pad_frac=0)
+        idx[1] = -1                      # a row without keys
+        idx[2, 0, 40:] = -1              # keys in the first split only
+        out, q, kv = _decode_call(wl, idx, seed, ws)
+        o = out.reshape(wl.batch, wl.H, wl.d_v)
+        assert (o[1] == 0).all(), "call %d: a row without keys must give 0" % call
+        check(wl, out, q, kv, idx, rows=np.array([r for r in range(wl.batch) if r != 1]))
