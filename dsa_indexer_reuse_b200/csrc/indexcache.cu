@@ -314,15 +314,11 @@ ic_status launch_indexer(const void* q_I, const float* q_scale, const void* w, i
         void* args[] = {&tm_q, &tm_k, &d};
         e = launch(pl.dec_kernel, dim3(grid), dim3(pl.dec_threads), pl.dec_smem, stream, args, pdl);
         if (e != cudaSuccess) return cuda_fail("decode indexer launch", e);
-        const int rows_smem = ic::TOPK_ROWS_SMEM;
-        e = cudaFuncSetAttribute(&ic::topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 ic::TOPK_ROWS_SMEM);
-        if (e != cudaSuccess) return cuda_fail("top-k rows smem attribute", e);
         const uint32_t* sc_ptr = d.scores;
         int stride = d.stride, n_vis = d.n_vis, kk = topk;
         void* rargs[] = {&sc_ptr, &stride, &n_vis, &kk, &idx_out};
-        e = launch(reinterpret_cast<const void*>(&ic::topk_rows_kernel), dim3(batch), dim3(ic::TOPK_ROWS_NT),
-                   rows_smem, stream, rargs, true);
+        e = launch(reinterpret_cast<const void*>(&ic::topk_rows_kernel), dim3(batch), dim3(ic::TOPK_ROWS_NT), 0,
+                   stream, rargs, true);
         if (e != cudaSuccess) return cuda_fail("top-k rows launch", e);
         return IC_OK;
     }

@@ -328,73 +328,176 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
     }
 }
 
-// Exact top-k of each score row written by indexer_decode_scores_kernel:
-// one 1024-thread CTA per row, the row staged in shared memory (dynamic).
-// A sample of one key in S (S = n_vis / 1024) gives a threshold tau, the
-// key just below the sample's r-th largest with r about 1.3 k / S, so about
-// 1.3 k keys of the row lie above it. The keys above tau are compacted in key
-// order and the exact select runs on those. When fewer than k or more than
-// TOPK_ROWS_PRE keys lie above tau, the exact select runs on the whole row
-// instead, so the result is exact either way. List position = key index
-// throughout, so ties go to the lower key; winners in ascending key order,
-// -1 padded.
+// Exact top-k of each score row written by indexer_decode_scores_kernel, by
+// radix select on the order-preserving score keys: one 1024-thread CTA per
+// row, thread t holding keys [32 t, 32 t + 32) in registers.
+//  * A block min / max gives the row's key range [kmin, kmax]; the select
+//    works on d = key - kmin, whose bit length nb is at most 32.
+//  * Each pass takes the next 12 (or fewer) bits of d below those already
+//    fixed: a shared-memory histogram of the keys that match the fixed high
+//    bits, then a block scan from the top finds the bin that holds the k-th
+//    largest key and how many keys of that bin are still to be taken. At most
+//    three passes fix every bit, giving the k-th largest key T exactly.
+//  * One scan of (keys > T, keys == T) per thread then writes the winners:
+//    every key above T and the lowest-indexed keys equal to T, in ascending
+//    key order. Ties thus go to the lower key; -1 pads rows with fewer than k
+//    visible keys.
 constexpr int TOPK_ROWS_NT = 1024;
 constexpr int TOPK_ROWS_E = 32;
 constexpr int TOPK_ROWS_MAX = TOPK_ROWS_NT * TOPK_ROWS_E;
-constexpr int TOPK_ROWS_PRE = 4 * TOPK_ROWS_NT;  // capacity of the pre-filtered list
-constexpr int TOPK_ROWS_SMEM = TOPK_ROWS_MAX * 4 + TOPK_ROWS_PRE * 8;
+constexpr int TOPK_RADIX_BITS = 12;
+constexpr int TOPK_RADIX_BINS = 1 << TOPK_RADIX_BITS;
+static_assert(TOPK_RADIX_BINS == 4 * TOPK_ROWS_NT, "four histogram bins per thread");
+
+// Inclusive sum over the 1024 threads of the block, in thread order; `total`
+// gets the block's sum. `red` is 32 words of shared memory, free again when
+// the call returns.
+__device__ __forceinline__ uint32_t block_scan_1024(uint32_t v, uint32_t* red, uint32_t& total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+    }
+    if (lane == 31) red[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t w = red[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t n = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += n;
+        }
+        red[lane] = w;
+    }
+    __syncthreads();
+    total = red[31];
+    const uint32_t before = warp > 0 ? red[warp - 1] : 0u;
+    __syncthreads();
+    return v + before;
+}
 
 __global__ void __launch_bounds__(TOPK_ROWS_NT)
     topk_rows_kernel(const uint32_t* __restrict__ scores, int stride, int n_vis, int topk,
                      int32_t* __restrict__ idx_out) {
-    __shared__ SelectScratch<TOPK_ROWS_NT, TOPK_ROWS_E> sc;
-    __shared__ SelectScratch<TOPK_ROWS_NT, 4> sc4;
-    __shared__ SelectScratch<TOPK_ROWS_NT, 1> sc1;
-    extern __shared__ uint4 rows_smem[];
-    uint32_t* skey = reinterpret_cast<uint32_t*>(rows_smem);
-    uint32_t* pkey = skey + TOPK_ROWS_MAX;
-    int32_t* pidx = reinterpret_cast<int32_t*>(pkey + TOPK_ROWS_PRE);
+    __shared__ uint32_t hist[TOPK_RADIX_BINS];
+    __shared__ uint32_t red[32];
+    __shared__ uint32_t mm[2][32];
+    __shared__ uint32_t pick[2];  // bin holding the k-th key, keys of it still to take
     const int row = blockIdx.x;
     const int tid = threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
     griddep_sync();  // the score rows come from the previous kernel
-    // stride is a multiple of 128 keys, so every row starts 16-byte aligned
-    const uint4* src = reinterpret_cast<const uint4*>(scores + static_cast<int64_t>(row) * stride);
-    for (int i = tid; i < (n_vis + 3) / 4; i += TOPK_ROWS_NT) rows_smem[i] = __ldg(src + i);
-    __syncthreads();
     int32_t* out = idx_out + static_cast<int64_t>(row) * topk;
-    auto emit_out = [&](int pos, uint32_t, int32_t iv) { out[pos] = iv; };
-    int kept = -1;
-    const int S = max(1, n_vis / TOPK_ROWS_NT);
-    const int ns = min(TOPK_ROWS_NT, (n_vis + S - 1) / S);
-    const int r = (13 * topk + 10 * S - 1) / (10 * S) + 8;
-    if (n_vis > topk && r < ns) {
-        const SelectResult samp = block_select<TOPK_ROWS_NT, 1>(
-            ns, r, true, r, 0u, tid, 1, sc1, [&](int pos) { return skey[pos * S]; }, [&](int pos) { return pos; },
-            [&](int, uint32_t, int32_t) {});
-        const uint32_t tau = samp.thr;
-        const int cnt = block_compact<TOPK_ROWS_NT, TOPK_ROWS_E>(
-            n_vis, tid, 1, sc, [&](int pos) { return skey[pos]; }, [&](int pos) { return pos; },
-            [&](uint32_t k) { return k > tau; }, [&](int c) { return c >= topk && c <= TOPK_ROWS_PRE; },
-            [&](int o, uint32_t kv, int32_t iv) {
-                if (o < TOPK_ROWS_PRE) {
-                    pkey[o] = kv;
-                    pidx[o] = iv;
-                }
-            });
-        if (cnt >= 0) {
-            kept = block_select<TOPK_ROWS_NT, 4>(cnt, topk, true, topk, 0u, tid, 1, sc4,
-                                                 [&](int pos) { return pkey[pos]; },
-                                                 [&](int pos) { return pidx[pos]; }, emit_out)
-                       .kept;
+    if (n_vis <= topk) {  // every visible key wins (uniform across the block)
+        for (int i = tid; i < topk; i += TOPK_ROWS_NT) out[i] = i < n_vis ? i : -1;
+        return;
+    }
+    // this thread's keys; stride is a multiple of 128 keys and at least n_vis,
+    // so a 32-key chunk that starts inside the row ends inside it too
+    const int i0 = tid * TOPK_ROWS_E;
+    const int nv = min(max(n_vis - i0, 0), TOPK_ROWS_E);  // its first nv keys are visible
+    uint32_t key[TOPK_ROWS_E];
+    if (nv > 0) {
+        const uint4* src = reinterpret_cast<const uint4*>(scores + static_cast<int64_t>(row) * stride + i0);
+#pragma unroll
+        for (int j = 0; j < TOPK_ROWS_E / 4; ++j) {
+            const uint4 v = __ldg(src + j);
+            key[4 * j] = v.x;
+            key[4 * j + 1] = v.y;
+            key[4 * j + 2] = v.z;
+            key[4 * j + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < TOPK_ROWS_E; ++j) key[j] = 0u;
+    }
+    // key range of the row
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+    for (int j = 0; j < TOPK_ROWS_E; ++j) {
+        if (j < nv) {
+            kmin = min(kmin, key[j]);
+            kmax = max(kmax, key[j]);
         }
     }
-    if (kept < 0) {
-        kept = block_select<TOPK_ROWS_NT, TOPK_ROWS_E>(n_vis, topk, true, topk, 0u, tid, 1, sc,
-                                                       [&](int pos) { return skey[pos]; },
-                                                       [&](int pos) { return pos; }, emit_out)
-                   .kept;
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (lane == 0) {
+        mm[0][warp] = kmin;
+        mm[1][warp] = kmax;
     }
-    for (int i = kept + tid; i < topk; i += TOPK_ROWS_NT) out[i] = -1;
+    __syncthreads();
+    kmin = __reduce_min_sync(0xffffffffu, mm[0][lane]);
+    kmax = __reduce_max_sync(0xffffffffu, mm[1][lane]);
+
+    // radix passes over d = key - kmin, high bits first
+    int hi = 32 - __clz(kmax - kmin);  // bits of d not fixed yet (0: every key equal)
+    uint32_t prefix = 0u;               // the fixed bits of the k-th largest d
+    uint32_t k_rem = static_cast<uint32_t>(topk);
+    while (hi > 0) {  // uniform across the block
+        const int lo = max(0, hi - TOPK_RADIX_BITS);
+        const uint32_t mask = (1u << (hi - lo)) - 1u;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) hist[4 * tid + q] = 0u;
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < TOPK_ROWS_E; ++j) {
+            const uint32_t d = key[j] - kmin;
+            if (j < nv && (static_cast<uint64_t>(d) >> hi) == prefix) atomicAdd(&hist[(d >> lo) & mask], 1u);
+        }
+        __syncthreads();
+        uint32_t h4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) h4[q] = hist[4 * tid + q];
+        const uint32_t mine = h4[0] + h4[1] + h4[2] + h4[3];
+        uint32_t total;
+        const uint32_t incl = block_scan_1024(mine, red, total);
+        uint32_t above = total - incl;  // keys in the bins of higher threads
+#pragma unroll
+        for (int q = 3; q >= 0; --q) {
+            if (above < k_rem && k_rem <= above + h4[q]) {
+                pick[0] = static_cast<uint32_t>(4 * tid + q);
+                pick[1] = k_rem - above;
+            }
+            above += h4[q];
+        }
+        __syncthreads();
+        prefix = (prefix << (hi - lo)) | pick[0];
+        k_rem = pick[1];
+        hi = lo;
+        __syncthreads();  // pick is rewritten by the next pass
+    }
+    const uint32_t T = kmin + prefix;  // the k-th largest key; k_rem keys equal to it win
+
+    // winners in key order: a packed scan of (keys above T, keys equal to T)
+    uint32_t gt = 0, eq = 0;
+#pragma unroll
+    for (int j = 0; j < TOPK_ROWS_E; ++j) {
+        if (j < nv) {
+            gt += key[j] > T ? 1u : 0u;
+            eq += key[j] == T ? 1u : 0u;
+        }
+    }
+    uint32_t total;
+    const uint32_t packed = (eq << 16) | gt;  // each half sums to at most 32768
+    const uint32_t excl = block_scan_1024(packed, red, total) - packed;
+    uint32_t tie = excl >> 16;
+    int pos = static_cast<int>((excl & 0xffffu) + min(tie, k_rem));
+#pragma unroll
+    for (int j = 0; j < TOPK_ROWS_E; ++j) {
+        if (j < nv) {
+            bool take = key[j] > T;
+            if (key[j] == T) {
+                take = tie < k_rem;
+                ++tie;
+            }
+            if (take) {
+                if (IC_DCHECK(pos < topk)) out[pos] = i0 + j;
+                ++pos;
+            }
+        }
+    }
 }
 
 }  // namespace ic

@@ -1,9 +1,9 @@
 """Exact parity of the decode path (one query per sequence, 64 heads,
 d_I = 128: score rows + per-row select) on inputs whose scores are exact in
 fp32, so indices must match the oracle bit for bit. Small-integer inputs give
-many exactly equal scores (ties to the lower key), all-equal scores force the
-select's fallback from its sampled threshold, and short contexts give fewer
-than k keys."""
+many exactly equal scores (ties to the lower key), all-equal scores leave the
+radix select no bit to fix, three distinct scores put the k-th key in a large
+class of equal keys, and short contexts give fewer than k keys."""
 
 import numpy as np
 import pytest
@@ -60,3 +60,21 @@ def test_decode_rows_all_equal_scores(cuda_ok):
     dev = torch.device("cuda")
     got = ic.indexer_topk(q.to(dev), w.to(dev), k.to(dev), topk, q_pos0=n_k - 1).cpu().numpy()
     assert np.array_equal(got.reshape(B, topk), np.tile(np.arange(topk, dtype=np.int32), (B, 1)))
+
+
+def test_decode_rows_three_distinct_scores(cuda_ok):
+    # every key row is one of three patterns, so each sequence has three
+    # distinct scores and the k-th largest sits in a class of ~11k equal keys:
+    # the radix select fixes every bit of that score and takes the class's
+    # lowest key indices (ties go to the lower key)
+    B, n_k, topk = 2, 32768, 2048
+    g = torch.Generator().manual_seed(9)
+    q = torch.randint(-3, 4, (B, 1, 64, 128), generator=g).to(torch.bfloat16)
+    w = torch.randint(-3, 4, (B, 1, 64), generator=g).to(torch.bfloat16)
+    pats = torch.randint(-3, 4, (B, 3, 128), generator=g).to(torch.bfloat16)
+    cls = torch.randint(0, 3, (B, n_k), generator=g)
+    k = torch.stack([pats[b][cls[b]] for b in range(B)])
+    dev = torch.device("cuda")
+    got = ic.indexer_topk(q.to(dev), w.to(dev), k.to(dev), topk, q_pos0=n_k - 1).cpu().numpy()
+    want = _oracle(q, w, k, topk, n_k - 1)
+    assert np.array_equal(canon(got.reshape(B, topk)), canon(want))
