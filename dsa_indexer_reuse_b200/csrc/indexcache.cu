@@ -317,8 +317,8 @@ ic_status launch_indexer(const void* q_I, const float* q_scale, const void* w, i
         const uint32_t* sc_ptr = d.scores;
         int stride = d.stride, n_vis = d.n_vis, kk = topk;
         void* rargs[] = {&sc_ptr, &stride, &n_vis, &kk, &idx_out};
-        e = launch(reinterpret_cast<const void*>(&ic::topk_rows_kernel), dim3(batch), dim3(ic::TOPK_ROWS_NT), 0,
-                   stream, rargs, true);
+        e = launch(reinterpret_cast<const void*>(&ic::topk_rows_kernel), dim3(batch * ic::TOPK_ROWS_CL),
+                   dim3(ic::TOPK_ROWS_NT), 0, stream, rargs, true);
         if (e != cudaSuccess) return cuda_fail("top-k rows launch", e);
         return IC_OK;
     }

@@ -27,6 +27,8 @@
 // warp 3 idle, warps 4-19 the epilogue warpgroups.
 #pragma once
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "topk_select.cuh"
 
@@ -329,25 +331,31 @@ __global__ void __launch_bounds__(Cfg::THREADS, 1)
 }
 
 // Exact top-k of each score row written by indexer_decode_scores_kernel, by
-// radix select on the order-preserving score keys: one 1024-thread CTA per
-// row, thread t holding keys [32 t, 32 t + 32) in registers.
-//  * A block min / max gives the row's key range [kmin, kmax]; the select
-//    works on d = key - kmin, whose bit length nb is at most 32.
+// radix select on the order-preserving score keys. A row belongs to one
+// cluster of TOPK_ROWS_CL CTAs: CTA c holds keys [8192 c, 8192 c + 8192),
+// thread t of it keys [8192 c + 8 t, 8192 c + 8 t + 8), in registers.
+//  * The cluster's min / max gives the row's key range [kmin, kmax]; the
+//    select works on d = key - kmin, whose bit length is at most 32.
 //  * Each pass takes the next 12 (or fewer) bits of d below those already
-//    fixed: a shared-memory histogram of the keys that match the fixed high
-//    bits, then a block scan from the top finds the bin that holds the k-th
-//    largest key and how many keys of that bin are still to be taken. At most
-//    three passes fix every bit, giving the k-th largest key T exactly.
-//  * One scan of (keys > T, keys == T) per thread then writes the winners:
-//    every key above T and the lowest-indexed keys equal to T, in ascending
-//    key order. Ties thus go to the lower key; -1 pads rows with fewer than k
-//    visible keys.
+//    fixed. Every CTA histograms its keys that match the fixed high bits in
+//    its own shared memory; each then sums the cluster's histograms through
+//    distributed shared memory and, with a block scan from the top, finds the
+//    bin that holds the k-th largest key and how many keys of that bin are
+//    still to be taken. Every CTA computes the same sums, so all take the same
+//    path. At most three passes fix every bit, giving the k-th largest key T.
+//  * A packed scan of (keys > T, keys == T) per thread, offset by the counts
+//    of the lower-ranked CTAs, then writes the winners: every key above T and
+//    the lowest-indexed keys equal to T, in ascending key order. Ties thus go
+//    to the lower key; -1 pads rows with fewer than k visible keys.
 constexpr int TOPK_ROWS_NT = 1024;
-constexpr int TOPK_ROWS_E = 32;
-constexpr int TOPK_ROWS_MAX = TOPK_ROWS_NT * TOPK_ROWS_E;
+constexpr int TOPK_ROWS_CL = 4;  // CTAs per row (one cluster)
+constexpr int TOPK_ROWS_E = 8;   // keys per thread
+constexpr int TOPK_ROWS_CTA = TOPK_ROWS_NT * TOPK_ROWS_E;
+constexpr int TOPK_ROWS_MAX = TOPK_ROWS_CL * TOPK_ROWS_CTA;
 constexpr int TOPK_RADIX_BITS = 12;
 constexpr int TOPK_RADIX_BINS = 1 << TOPK_RADIX_BITS;
 static_assert(TOPK_RADIX_BINS == 4 * TOPK_ROWS_NT, "four histogram bins per thread");
+static_assert(TOPK_ROWS_MAX == 32768, "rows of up to 32768 keys");
 
 // Inclusive sum over the 1024 threads of the block, in thread order; `total`
 // gets the block's sum. `red` is 32 words of shared memory, free again when
@@ -377,25 +385,32 @@ __device__ __forceinline__ uint32_t block_scan_1024(uint32_t v, uint32_t* red, u
     return v + before;
 }
 
-__global__ void __launch_bounds__(TOPK_ROWS_NT)
+__global__ void __cluster_dims__(TOPK_ROWS_CL, 1, 1) __launch_bounds__(TOPK_ROWS_NT)
     topk_rows_kernel(const uint32_t* __restrict__ scores, int stride, int n_vis, int topk,
                      int32_t* __restrict__ idx_out) {
-    __shared__ uint32_t hist[TOPK_RADIX_BINS];
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    __shared__ __align__(16) uint32_t hist[TOPK_RADIX_BINS];
     __shared__ uint32_t red[32];
     __shared__ uint32_t mm[2][32];
     __shared__ uint32_t pick[2];  // bin holding the k-th key, keys of it still to take
-    const int row = blockIdx.x;
+    // read by the other CTAs of the cluster: this CTA's key min and max, and
+    // its packed count of (keys == T) << 16 | (keys > T)
+    __shared__ uint32_t xch[3];
+    const int crank = static_cast<int>(cluster.block_rank());
+    const int row = blockIdx.x / TOPK_ROWS_CL;
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
     griddep_sync();  // the score rows come from the previous kernel
     int32_t* out = idx_out + static_cast<int64_t>(row) * topk;
-    if (n_vis <= topk) {  // every visible key wins (uniform across the block)
-        for (int i = tid; i < topk; i += TOPK_ROWS_NT) out[i] = i < n_vis ? i : -1;
+    if (n_vis <= topk) {  // every visible key wins (uniform across the cluster)
+        for (int i = crank * TOPK_ROWS_NT + tid; i < topk; i += TOPK_ROWS_CL * TOPK_ROWS_NT)
+            out[i] = i < n_vis ? i : -1;
         return;
     }
     // this thread's keys; stride is a multiple of 128 keys and at least n_vis,
-    // so a 32-key chunk that starts inside the row ends inside it too
-    const int i0 = tid * TOPK_ROWS_E;
+    // so an 8-key chunk that starts inside the row ends inside it too
+    const int i0 = crank * TOPK_ROWS_CTA + tid * TOPK_ROWS_E;
     const int nv = min(max(n_vis - i0, 0), TOPK_ROWS_E);  // its first nv keys are visible
     uint32_t key[TOPK_ROWS_E];
     if (nv > 0) {
@@ -412,7 +427,7 @@ __global__ void __launch_bounds__(TOPK_ROWS_NT)
 #pragma unroll
         for (int j = 0; j < TOPK_ROWS_E; ++j) key[j] = 0u;
     }
-    // key range of the row
+    // key range of the row: this CTA's, then the cluster's
     uint32_t kmin = 0xffffffffu, kmax = 0u;
 #pragma unroll
     for (int j = 0; j < TOPK_ROWS_E; ++j) {
@@ -428,14 +443,29 @@ __global__ void __launch_bounds__(TOPK_ROWS_NT)
         mm[1][warp] = kmax;
     }
     __syncthreads();
-    kmin = __reduce_min_sync(0xffffffffu, mm[0][lane]);
-    kmax = __reduce_max_sync(0xffffffffu, mm[1][lane]);
+    if (warp == 0) {
+        kmin = __reduce_min_sync(0xffffffffu, mm[0][lane]);
+        kmax = __reduce_max_sync(0xffffffffu, mm[1][lane]);
+        if (lane == 0) {
+            xch[0] = kmin;
+            xch[1] = kmax;
+        }
+    }
+    cluster.sync();
+    kmin = 0xffffffffu;
+    kmax = 0u;
+#pragma unroll
+    for (int c = 0; c < TOPK_ROWS_CL; ++c) {
+        const uint32_t* x = cluster.map_shared_rank(xch, c);
+        kmin = min(kmin, x[0]);
+        kmax = max(kmax, x[1]);
+    }
 
     // radix passes over d = key - kmin, high bits first
     int hi = 32 - __clz(kmax - kmin);  // bits of d not fixed yet (0: every key equal)
     uint32_t prefix = 0u;               // the fixed bits of the k-th largest d
     uint32_t k_rem = static_cast<uint32_t>(topk);
-    while (hi > 0) {  // uniform across the block
+    while (hi > 0) {  // uniform across the cluster
         const int lo = max(0, hi - TOPK_RADIX_BITS);
         const uint32_t mask = (1u << (hi - lo)) - 1u;
 #pragma unroll
@@ -446,13 +476,18 @@ __global__ void __launch_bounds__(TOPK_ROWS_NT)
             const uint32_t d = key[j] - kmin;
             if (j < nv && (static_cast<uint64_t>(d) >> hi) == prefix) atomicAdd(&hist[(d >> lo) & mask], 1u);
         }
-        __syncthreads();
-        uint32_t h4[4];
+        cluster.sync();  // every CTA's histogram is complete
+        uint32_t h4[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) h4[q] = hist[4 * tid + q];
-        const uint32_t mine = h4[0] + h4[1] + h4[2] + h4[3];
+        for (int c = 0; c < TOPK_ROWS_CL; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(cluster.map_shared_rank(hist, c) + 4 * tid);
+            h4[0] += v.x;
+            h4[1] += v.y;
+            h4[2] += v.z;
+            h4[3] += v.w;
+        }
         uint32_t total;
-        const uint32_t incl = block_scan_1024(mine, red, total);
+        const uint32_t incl = block_scan_1024(h4[0] + h4[1] + h4[2] + h4[3], red, total);
         uint32_t above = total - incl;  // keys in the bins of higher threads
 #pragma unroll
         for (int q = 3; q >= 0; --q) {
@@ -466,11 +501,13 @@ __global__ void __launch_bounds__(TOPK_ROWS_NT)
         prefix = (prefix << (hi - lo)) | pick[0];
         k_rem = pick[1];
         hi = lo;
-        __syncthreads();  // pick is rewritten by the next pass
+        // the next pass rewrites hist, which the other CTAs read above, and pick
+        cluster.sync();
     }
     const uint32_t T = kmin + prefix;  // the k-th largest key; k_rem keys equal to it win
 
-    // winners in key order: a packed scan of (keys above T, keys equal to T)
+    // winners in key order: a packed scan of (keys above T, keys equal to T),
+    // offset by the packed counts of the lower-ranked CTAs
     uint32_t gt = 0, eq = 0;
 #pragma unroll
     for (int j = 0; j < TOPK_ROWS_E; ++j) {
@@ -480,8 +517,11 @@ __global__ void __launch_bounds__(TOPK_ROWS_NT)
         }
     }
     uint32_t total;
-    const uint32_t packed = (eq << 16) | gt;  // each half sums to at most 32768
-    const uint32_t excl = block_scan_1024(packed, red, total) - packed;
+    const uint32_t packed = (eq << 16) | gt;  // each half sums to at most 32768 over the row
+    uint32_t excl = block_scan_1024(packed, red, total) - packed;
+    if (tid == 0) xch[2] = total;
+    cluster.sync();
+    for (int c = 0; c < crank; ++c) excl += cluster.map_shared_rank(xch, c)[2];
     uint32_t tie = excl >> 16;
     int pos = static_cast<int>((excl & 0xffffu) + min(tie, k_rem));
 #pragma unroll
@@ -498,6 +538,7 @@ __global__ void __launch_bounds__(TOPK_ROWS_NT)
             }
         }
     }
+    cluster.sync();  // no CTA leaves while another may still read its xch
 }
 
 }  // namespace ic
