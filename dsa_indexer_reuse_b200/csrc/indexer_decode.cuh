@@ -390,7 +390,10 @@ __global__ void __cluster_dims__(TOPK_ROWS_CL, 1, 1) __launch_bounds__(TOPK_ROWS
                      int32_t* __restrict__ idx_out) {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
-    __shared__ __align__(16) uint32_t hist[TOPK_RADIX_BINS];
+    // two histograms, alternating between passes: a CTA rewrites one only
+    // after every CTA of the cluster has passed the next pass's barrier, so
+    // after the last remote read of it
+    __shared__ __align__(16) uint32_t hist2[2][TOPK_RADIX_BINS];
     __shared__ uint32_t red[32];
     __shared__ uint32_t mm[2][32];
     __shared__ uint32_t pick[2];  // bin holding the k-th key, keys of it still to take
@@ -465,7 +468,9 @@ __global__ void __cluster_dims__(TOPK_ROWS_CL, 1, 1) __launch_bounds__(TOPK_ROWS
     int hi = 32 - __clz(kmax - kmin);  // bits of d not fixed yet (0: every key equal)
     uint32_t prefix = 0u;               // the fixed bits of the k-th largest d
     uint32_t k_rem = static_cast<uint32_t>(topk);
+    int npass = 0;
     while (hi > 0) {  // uniform across the cluster
+        uint32_t* hist = hist2[npass++ & 1];
         const int lo = max(0, hi - TOPK_RADIX_BITS);
         const uint32_t mask = (1u << (hi - lo)) - 1u;
 #pragma unroll
@@ -501,8 +506,7 @@ __global__ void __cluster_dims__(TOPK_ROWS_CL, 1, 1) __launch_bounds__(TOPK_ROWS
         prefix = (prefix << (hi - lo)) | pick[0];
         k_rem = pick[1];
         hi = lo;
-        // the next pass rewrites hist, which the other CTAs read above, and pick
-        cluster.sync();
+        __syncthreads();  // pick is rewritten by the next pass
     }
     const uint32_t T = kmin + prefix;  // the k-th largest key; k_rem keys equal to it win
 
