@@ -272,6 +272,8 @@ ic_status launch_indexer(const void* q_I, const float* q_scale, const void* w, i
                                     d_I, topk, idx_out);
     if (st != IC_OK) return st;
     if (batch == 0 || n_q == 0) return IC_OK;
+    // the scratch holds 256-byte aligned sub-arrays read with vector loads
+    if (ws != nullptr && !aligned256(ws)) return IC_ERR_WORKSPACE;
     IdxPlan pl;
     if (!choose_idx_plan(H_I, d_I, qk_dt, n_q, &pl)) return IC_ERR_UNSUPPORTED;
     if (!plan_supports_topk(pl, topk)) return IC_ERR_UNSUPPORTED;
@@ -442,6 +444,8 @@ ic_status launch_attn(const void* q, const void* kv, const int32_t* idx, int bat
     if (batch == 0 || n_q == 0) return IC_OK;
     if (!q || !idx || !out || (n_k > 0 && !kv)) return IC_ERR_INVALID_ARG;
     if (!aligned16(q) || (n_k > 0 && !aligned16(kv))) return IC_ERR_INVALID_ARG;
+    // the split partials are 256-byte aligned sub-arrays read with vector loads
+    if (ws != nullptr && !aligned256(ws)) return IC_ERR_WORKSPACE;
     AttnPlan pl;
     if (!choose_attn_plan(d_qk, d_v, &pl)) return IC_ERR_UNSUPPORTED;
     if (H > 64 || topk > ic::AttnCfg<64, 64>::MAX_TOPK) return IC_ERR_UNSUPPORTED;

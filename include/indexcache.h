@@ -20,7 +20,8 @@
  *    owned by the caller (ic_layer_stack_host also takes host pointers). The
  *    library never allocates device memory; calls
  *    that need scratch take a caller-provided workspace whose size the
- *    matching *_workspace_size function reports.
+ *    matching *_workspace_size function reports. A workspace pointer, when
+ *    not NULL, must be 256-byte aligned (IC_ERR_WORKSPACE otherwise).
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream). Work is enqueued asynchronously; no call synchronises, so the
  *    launching calls may be captured into a CUDA graph.

@@ -100,6 +100,11 @@ def test_invalid_calls_fail_on_host(ic):
                             None, 0, None) == 1
     assert L.ic_sparse_attn(fake, fake, fake, 1, 4, 16, 8, 576, 512, 8, ctypes.c_float(0.1), None,
                             None, 0, None) == 1
+    # a workspace that is not 256-byte aligned is refused before any device work
+    assert L.ic_indexer_topk(fake, None, fake, 0, fake, None, 0, 1, 1, 16, 15, 64, 128, 8, fake,
+                             P(0x10010), 1 << 20, None) == 6
+    assert L.ic_sparse_attn(fake, fake, fake, 1, 1, 16, 8, 576, 512, 8, ctypes.c_float(0.1), fake,
+                            P(0x10010), 1 << 20, None) == 6
     # empty problems are valid no-ops
     assert L.ic_indexer_topk(None, None, None, 0, None, None, 0, 0, 0, 0, 0, 64, 128, 8, None,
                              None, 0, None) == 0
